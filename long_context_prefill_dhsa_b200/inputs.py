@@ -1,0 +1,219 @@
+"""Seeded synthetic inputs for the DHSA prefill path.
+
+This module is shared by the CPU oracle's tests and by the CUDA path's tests
+and benchmark. It holds only the recipe that draws the inputs -- chunk
+layouts, Q/K/V values, needle plants -- and none of the method's arithmetic
+(no pooling, scoring, selection or attention).
+
+Workloads follow the five layer shapes of the DHSA README's "Kernel-level
+Latency" section (Llama-3.1-8B and Qwen2.5-3B attention layers, head dim 128,
+BF16) with synthetic values standing in for real activations:
+
+* chunk lengths are drawn i.i.d. until they cover L, and the last chunk is
+  truncated to fit;
+* a Q (K) row is its chunk's per-head mean vector mu ~ N(0, I) plus
+  0.5 * N(0, I) noise, V ~ N(0, 1);
+* the ragged stress workload plants "needles": a K chunk mean set to 3x the
+  mean of a later query chunk of a head in the same GQA group, a synthetic
+  stand-in for the Needle-in-a-Haystack retrieval test.
+
+Every (tensor, batch, head) draws from its own counter-derived NumPy stream
+(`SeedSequence([seed, workload_id, tag, b, h])`), so any head can be rebuilt
+alone, e.g. for sampled checks at full size. Values are drawn in float32 and
+rounded to bfloat16 (round to nearest even); bf16 tensors are carried as raw
+uint16 bit patterns.
+"""
+from __future__ import annotations
+
+import dataclasses
+from typing import Optional
+
+import numpy as np
+
+HEAD_DIM = 128
+
+# stream tags
+_TAG_LEN, _TAG_Q, _TAG_K, _TAG_V, _TAG_NEEDLE = 0, 1, 2, 3, 4
+
+
+@dataclasses.dataclass(frozen=True)
+class Workload:
+    """One synthetic attention layer."""
+    wid: int                 # workload id; part of every stream's seed
+    name: str
+    B: int
+    Hq: int
+    Hkv: int
+    L: int
+    length_kind: str         # "uniform" or "geometric"
+    length_lo: int
+    length_hi: int
+    length_mean: float = 0.0  # geometric only
+    k: int = 8               # earlier chunks kept per query chunk (besides the diagonal)
+    needles_per_head: int = 0
+    seed: int = 0
+    target_density: Optional[float] = None
+
+    @property
+    def G(self) -> int:
+        return self.Hq // self.Hkv
+
+    def with_(self, **kw) -> "Workload":
+        return dataclasses.replace(self, **kw)
+
+
+# The five layer workloads. k for the three density-targeted ones is the
+# smallest k whose kept density (kept token pairs / causal pairs, averaged over
+# (b, hq)) on these seeded inputs reaches the target; the values were found by
+# oracle/freeze_k.py, which runs the CPU oracle only.
+WORKLOADS = {
+    "tiny": Workload(1, "tiny-2k", 1, 2, 1, 2048, "uniform", 16, 64, k=8),
+    "qwen3b-8k": Workload(2, "qwen2.5-3b-8k", 1, 16, 2, 8192, "uniform", 32, 128,
+                          k=10, target_density=0.20),
+    "llama8b-32k": Workload(3, "llama3.1-8b-32k", 1, 32, 8, 32768, "uniform", 32, 256,
+                            k=10, target_density=0.10),
+    "llama8b-128k": Workload(4, "llama3.1-8b-128k", 1, 32, 8, 131072, "uniform", 64, 256,
+                             k=17, target_density=0.05),
+    "ragged-64k": Workload(5, "ragged-needles-64k", 2, 32, 8, 65536, "geometric", 1, 1024,
+                           length_mean=96.0, k=32, needles_per_head=16),
+}
+
+
+def _rng(w: Workload, *tags: int) -> np.random.Generator:
+    return np.random.default_rng(np.random.SeedSequence([w.seed, w.wid, *tags]))
+
+
+def chunk_lengths(w: Workload, b: int) -> np.ndarray:
+    """Chunk lengths of batch element b: i.i.d. draws until they cover L.
+
+    A batch of draws large enough to cover L is taken from the stream at once;
+    the prefix up to the first draw whose running sum reaches L is kept and the
+    last kept length is cut to L - (sum of the previous ones), so it is >= 1.
+    """
+    rng = _rng(w, _TAG_LEN, b)
+    n_draw = w.L // max(1, w.length_lo) + 2
+    if w.length_kind == "uniform":
+        lens = rng.integers(w.length_lo, w.length_hi + 1, size=n_draw)
+    elif w.length_kind == "geometric":
+        lens = rng.geometric(1.0 / w.length_mean, size=n_draw)
+        lens = np.clip(lens, w.length_lo, w.length_hi)
+    else:
+        raise ValueError(w.length_kind)
+    csum = np.cumsum(lens)
+    n = int(np.searchsorted(csum, w.L)) + 1          # first index with csum >= L
+    lens = lens[:n].astype(np.int64)
+    lens[-1] = w.L - (csum[n - 2] if n > 1 else 0)
+    assert lens.sum() == w.L and lens.min() >= 1
+    return lens
+
+
+def offsets(w: Workload):
+    """int32 off[B][Nmax+1] (padded with L) and int32 n_chunks[B]."""
+    lens = [chunk_lengths(w, b) for b in range(w.B)]
+    nmax = max(len(x) for x in lens)
+    off = np.full((w.B, nmax + 1), w.L, dtype=np.int32)
+    for b, x in enumerate(lens):
+        off[b, 0] = 0
+        off[b, 1:len(x) + 1] = np.cumsum(x)
+    n_chunks = np.array([len(x) for x in lens], dtype=np.int32)
+    return off, n_chunks
+
+
+def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
+    """Round float32 to bfloat16 (nearest, ties to even); returns uint16 bits."""
+    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32)
+    bias = ((u >> 16) & 1) + np.uint32(0x7FFF)
+    return ((u + bias) >> 16).astype(np.uint16)
+
+
+def bf16_bits_to_f32(u: np.ndarray) -> np.ndarray:
+    return (u.astype(np.uint32) << 16).view(np.float32)
+
+
+def _chunk_ids(off_b: np.ndarray, n: int, L: int) -> np.ndarray:
+    lens = np.diff(off_b[: n + 1])
+    return np.repeat(np.arange(n), lens)
+
+
+def _mu_q(w: Workload, b: int, hq: int, n: int) -> np.ndarray:
+    return _rng(w, _TAG_Q, b, hq).standard_normal((n, HEAD_DIM), dtype=np.float32)
+
+
+def needles(w: Workload, n_chunks: np.ndarray):
+    """Planted pairs: list per b of (hq, i, j) with j < i and i > k.
+
+    For each query head, `needles_per_head` query chunks i are drawn uniformly
+    from (k, N_b) and a key chunk j uniformly from [0, i), redrawing j until it
+    is distinct from every j already planted in the same kv head.
+    """
+    out = []
+    for b in range(w.B):
+        plants = []
+        if w.needles_per_head:
+            n = int(n_chunks[b])
+            if n <= w.k + 1:
+                raise ValueError("too few chunks to plant needles beyond k")
+            rng = _rng(w, _TAG_NEEDLE, b)
+            used = [set() for _ in range(w.Hkv)]
+            for hq in range(w.Hq):
+                hkv = hq // w.G
+                for _ in range(w.needles_per_head):
+                    i = int(rng.integers(w.k + 1, n))
+                    while True:
+                        j = int(rng.integers(0, i))
+                        if j not in used[hkv]:
+                            break
+                    used[hkv].add(j)
+                    plants.append((hq, i, j))
+        out.append(plants)
+    return out
+
+
+def make_inputs(w: Workload, heads_q=None, heads_kv=None, with_v=True):
+    """Build one workload.
+
+    Returns a dict with uint16 (bf16 bits) arrays Q[B,Hq,L,128],
+    K[B,Hkv,L,128], V[B,Hkv,L,128], int32 off[B][Nmax+1], int32 n_chunks[B]
+    and the needle list. `heads_q` / `heads_kv` restrict which heads are
+    filled (the rest stay zero), for sampled checks on large workloads;
+    `with_v=False` leaves V zero (routing only needs Q and K).
+    """
+    off, n_chunks = offsets(w)
+    plants = needles(w, n_chunks)
+    hq_set = range(w.Hq) if heads_q is None else heads_q
+    hkv_set = range(w.Hkv) if heads_kv is None else heads_kv
+    Q = np.zeros((w.B, w.Hq, w.L, HEAD_DIM), dtype=np.uint16)
+    K = np.zeros((w.B, w.Hkv, w.L, HEAD_DIM), dtype=np.uint16)
+    V = np.zeros((w.B, w.Hkv, w.L, HEAD_DIM), dtype=np.uint16)
+    for b in range(w.B):
+        n = int(n_chunks[b])
+        cid = _chunk_ids(off[b], n, w.L)
+        for hq in hq_set:
+            rng = _rng(w, _TAG_Q, b, hq)
+            mu = rng.standard_normal((n, HEAD_DIM), dtype=np.float32)
+            noise = rng.standard_normal((w.L, HEAD_DIM), dtype=np.float32)
+            noise *= np.float32(0.5)
+            noise += mu[cid]
+            Q[b, hq] = f32_to_bf16_bits(noise)
+        for hkv in hkv_set:
+            rng = _rng(w, _TAG_K, b, hkv)
+            mu = rng.standard_normal((n, HEAD_DIM), dtype=np.float32)
+            for (hq, i, j) in plants[b]:
+                if hq // w.G == hkv:
+                    mu[j] = np.float32(3.0) * _mu_q(w, b, hq, n)[i]
+            noise = rng.standard_normal((w.L, HEAD_DIM), dtype=np.float32)
+            noise *= np.float32(0.5)
+            noise += mu[cid]
+            K[b, hkv] = f32_to_bf16_bits(noise)
+            if not with_v:
+                continue
+            rng = _rng(w, _TAG_V, b, hkv)
+            V[b, hkv] = f32_to_bf16_bits(rng.standard_normal((w.L, HEAD_DIM), dtype=np.float32))
+    return dict(Q=Q, K=K, V=V, off=off, n_chunks=n_chunks, needles=plants, workload=w)
+
+
+def custom(B=1, Hq=2, Hkv=1, L=256, lo=1, hi=64, kind="uniform", mean=0.0, k=4,
+           seed=0, wid=100, needles_per_head=0, name="custom") -> Workload:
+    """A small workload for edge cases (ragged tails, one-row chunks, ...)."""
+    return Workload(wid, name, B, Hq, Hkv, L, kind, lo, hi, length_mean=mean, k=k,
+                    needles_per_head=needles_per_head, seed=seed)
