@@ -1,0 +1,397 @@
+"""Benchmark of one DHSA prefill layer (mask construction + sparse attention).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+A step is one pass of the whole hot path on one synthetic layer: pool(Q),
+pool(K), chunk score + top-k, block-CSR build and the sparse attention
+kernel, all on one stream, inputs resident in HBM. At N = 1 the workload is
+the 128K Llama-3.1-8B-shaped layer (the context length the metric is quoted
+at). With N > 1 (torchrun, one process per GPU) every rank runs its own
+independent layer: DHSA shards by head groups with no exchange, so ranks are
+replicas and the scaling is weak.
+
+Prints one JSON line on rank 0. `value` = amortised ms per layer over the
+whole job (max-over-ranks device time of K steps / (K * N)).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "ms per layer (mask+attn) and TFLOP/s on kept pairs at 128K, % of roofline"
+PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS = 6650.0, 1590.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="llama8b-128k")
+    ap.add_argument("--impl", default="dhsa", choices=["dhsa", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    return ap.parse_args()
+
+
+def peaks():
+    try:
+        p = json.load(open(PEAKS_PATH))
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
+
+
+# ----------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi clock / throttle samples while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.th = threading.Thread(target=self._read, daemon=True)
+            self.th.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------- helpers
+def kept_pair_count(off, n_chunks, sel, n_sel):
+    """Kept token pairs of the layer from the GPU selection (host arithmetic)."""
+    import torch
+    B, Hq, nmax, stride = sel.shape
+    lens = torch.diff(off.long(), dim=1)                                 # [B, Nmax]
+    total = 0
+    for b in range(B):
+        n = int(n_chunks[b])
+        lb = lens[b, :n]
+        s = sel[b, :, :n].long()
+        valid = s >= 0
+        lj = torch.where(valid, lb[s.clamp(min=0)], torch.zeros_like(s))
+        row_keys = lj.sum(-1) - lb[None, :]                               # earlier kept chunks
+        total += int((lb[None, :] * row_keys).sum() + (Hq * (lb * (lb + 1) // 2).sum()))
+    return total
+
+
+def routing_bytes(w, nmax, k):
+    """Algorithmic HBM bytes of the routing stages (one layer)."""
+    d = 128
+    x = w.B * (w.Hq + w.Hkv) * w.L * d * 2                 # read Q and K once
+    pooled = w.B * (w.Hq + w.Hkv) * nmax * d * 4           # write Qp/Kp
+    reread = pooled                                         # read them again for scoring
+    stride = min(k, nmax - 1) + 1
+    sel = w.B * w.Hq * nmax * (stride + 1) * 4 * 2          # write sel/n_sel, read in CSR build
+    csr = w.B * w.Hq * nmax * (stride + 3) * 4              # row_ptr, col_idx, cost
+    return x + pooled + reread + sel + csr
+
+
+def attn_bytes(w):
+    """Compulsory attention HBM bytes: Q, K, V read once, O written once."""
+    return w.B * (2 * w.Hq + 2 * w.Hkv) * w.L * 128 * 2
+
+
+# ----------------------------------------------------------------- oracle (CPU) leg
+def cpu_oracle_sample(d, w, seconds):
+    """Time the CPU oracle on a bounded sample of the layer and extrapolate
+    to ms per layer. Sample: pooling of one query head + its kv head, the
+    chunk scores/selection of that head, and the attention of as many of its
+    query chunks (in a fixed shuffled order) as fit in the time budget."""
+    from oracle import dhsa as ora
+    off, nc = d["off"], d["n_chunks"]
+    nmax = off.shape[1] - 1
+    cores = len(os.sched_getaffinity(0))
+    t0 = time.perf_counter()
+    Qp = ora.chunk_pool(ora.bf16_to_f64(d["Q"][:, :1]), off, nc, nmax)
+    Kp = ora.chunk_pool(ora.bf16_to_f64(d["K"][:, :1]), off, nc, nmax)
+    t_pool = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    S = ora.chunk_scores(Qp, Kp, nc)
+    sel = ora.select(S, nc, w.k)
+    t_route = time.perf_counter() - t0
+    Q = ora.bf16_to_f64(d["Q"][0, 0]).astype(np.float32)
+    K = ora.bf16_to_f64(d["K"][0, 0]).astype(np.float32)
+    V = ora.bf16_to_f64(d["V"][0, 0]).astype(np.float32)
+    n = int(nc[0])
+    order = np.random.default_rng(0).permutation(n)
+    done, t_attn = 0, 0.0
+    t0 = time.perf_counter()
+    for i in order:
+        ora.attn_chunk(Q, K, V, off[0], sel[0][0][i], int(i), 1.0 / math.sqrt(128), np.float32)
+        done += 1
+        t_attn = time.perf_counter() - t0
+        if t_attn > seconds:
+            break
+    heads = w.B * w.Hq
+    kv_frac = w.Hkv / w.Hq
+    est = (t_pool * (1 + kv_frac) / 2 * heads + t_route * heads + t_attn * (n / done) * heads)
+    return {"value": est * 1e3, "unit": "ms", "cores": cores, "kind": "oracle",
+            "sample": (f"oracle on (b=0, hq=0): pooling of Q and K, all {n} score/top-k rows, attention of "
+                       f"{done}/{n} query chunks; extrapolated x{heads} heads"
+                       f"{' x' + str(round(n / done, 2)) + ' chunks' if done < n else ''}")}
+
+
+# ----------------------------------------------------------------- reference arm
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from long_context_prefill_dhsa_b200 import inputs as I
+    w = I.WORKLOADS[args.workload]
+    d = I.make_inputs(w)
+    for _ in range(args.warmup):
+        cpu_oracle_sample(d, w, min(2.0, args.cpu_seconds))
+    vals = []
+    res = None
+    for _ in range(args.steps):
+        res = cpu_oracle_sample(d, w, args.cpu_seconds / max(1, args.steps))
+        vals.append(res["value"])
+    v = statistics.median(vals)
+    res["value"] = v
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "ms", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": v, "higher_is_better": False,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "L": w.L, "k": w.k,
+                   "chunk_len": f"{w.length_kind}[{w.length_lo},{w.length_hi}]"},
+        "cpu_baseline": res, "e2e": {"value": v, "unit": "ms", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+# ----------------------------------------------------------------- main arm
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+
+    from long_context_prefill_dhsa_b200 import binding, inputs as I
+    binding.load()
+    w = I.WORKLOADS[args.workload]
+    d = I.make_inputs(w)
+    dev = torch.device("cuda", local)
+    host = {x: torch.from_numpy(d[x]).view(torch.bfloat16).pin_memory() for x in "QKV"}
+    host_off = torch.from_numpy(d["off"]).pin_memory()
+    host_nc = torch.from_numpy(d["n_chunks"]).pin_memory()
+    Q, K, V = (host[x].to(dev) for x in "QKV")
+    off, nc = host_off.to(dev), host_nc.to(dev)
+    layer = binding.DHSAPrefill(w.B, w.Hq, w.Hkv, w.L, off, nc, w.k, device=dev)
+    stream = torch.cuda.current_stream()
+
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    n_launch_per_step = 7   # pool x2, score/top-k, CSR scan + fill, work list + attention
+
+    def step(timed_stages=None):
+        if timed_stages is None:
+            return layer.run(Q, K, V)
+        e0, e1, e2 = ev(), ev(), ev()
+        e0.record(stream)
+        layer.routing(Q, K)
+        e1.record(stream)
+        layer.attention(Q, K, V)
+        e2.record(stream)
+        timed_stages.append((e0, e1, e2))
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    binding.check_device_status()
+
+    stages = []
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        t0, t1 = ev(), ev()
+        t0.record(stream)
+        for _ in range(args.steps):
+            step(stages)
+        t1.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    total_ms = t0.elapsed_time(t1)
+    if world > 1:
+        tt = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        total_ms = float(tt.item())
+    flags = binding.check_device_status()
+    route_ms = statistics.median(a.elapsed_time(b) for a, b, _ in stages)
+    attn_ms = statistics.median(b.elapsed_time(c) for _, b, c in stages)
+    ms_step = total_ms / args.steps
+
+    nmax = d["off"].shape[1] - 1
+    pairs = kept_pair_count(off.cpu(), nc.cpu(), layer.sel.cpu(), layer.n_sel.cpu())
+    flop = 4.0 * 128 * pairs
+    hbm_peak, tc_peak, peak_kind = peaks()
+    attn_tflops = flop / (attn_ms * 1e-3) / 1e12
+    rbytes = routing_bytes(w, nmax, w.k)
+
+    # end to end through the public API with host buffers (pinned), on this rank
+    e2e = None
+    if not args.no_e2e:
+        out_host = torch.empty(host["Q"].shape, dtype=torch.bfloat16).pin_memory()
+        h2d = sum(host[x].numel() * 2 for x in "QKV") + host_off.numel() * 4 + host_nc.numel() * 4
+        d2h = out_host.numel() * 2
+
+        def e2e_step():
+            for x, dst in zip("QKV", (Q, K, V)):
+                dst.copy_(host[x], non_blocking=True)
+            off.copy_(host_off, non_blocking=True)
+            nc.copy_(host_nc, non_blocking=True)
+            O = layer.run(Q, K, V)
+            out_host.copy_(O, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        a, b = ev(), ev()
+        a.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = a.elapsed_time(b) / args.steps
+        if world > 1:
+            tt = torch.tensor([e2e_ms], device=dev)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            e2e_ms = float(tt.item())
+        e2e = {"value": e2e_ms / world, "unit": "ms", "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+
+    # dense comparisons (not part of the timed value): the same kernels with
+    # k = all causal chunks, and torch SDPA dense causal attention
+    dense = {}
+    if not args.no_dense and rank == 0:
+        try:
+            dl = binding.DHSAPrefill(w.B, w.Hq, w.Hkv, w.L, off, nc, 1 << 30, device=dev)
+            dl.run(Q, K, V)
+            torch.cuda.synchronize()
+            a, b = ev(), ev()
+            a.record(stream)
+            dl.run(Q, K, V)
+            b.record(stream)
+            torch.cuda.synchronize()
+            dense["dhsa_k_all_ms"] = a.elapsed_time(b)
+            del dl
+            import torch.nn.functional as F
+            Kr = K.repeat_interleave(w.G, dim=1)
+            Vr = V.repeat_interleave(w.G, dim=1)
+            F.scaled_dot_product_attention(Q, Kr, Vr, is_causal=True)
+            torch.cuda.synchronize()
+            a, b = ev(), ev()
+            a.record(stream)
+            F.scaled_dot_product_attention(Q, Kr, Vr, is_causal=True)
+            b.record(stream)
+            torch.cuda.synchronize()
+            dense["torch_sdpa_causal_ms"] = a.elapsed_time(b)
+            dense["speedup_vs_sdpa"] = dense["torch_sdpa_causal_ms"] / ms_step
+            dense["speedup_vs_k_all"] = dense["dhsa_k_all_ms"] / ms_step
+        except Exception as e:  # measurement only; never fails the bench
+            dense["error"] = repr(e)[:200]
+
+    cpu = None
+    if not args.no_cpu and rank == 0 and world == 1:
+        cpu = cpu_oracle_sample(d, w, args.cpu_seconds)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": ms_step / world, "unit": "ms", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": False, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "L": w.L, "head_dim": 128,
+                       "k": w.k, "chunk_len": f"{w.length_kind}[{w.length_lo},{w.length_hi}]", "n_chunks": nmax,
+                       "kept_density": pairs / (w.B * w.Hq * w.L * (w.L + 1) / 2),
+                       "parallelism": f"replicas x{world} (independent layers, no collective)",
+                       "l2": "inputs larger than L2 (Q+K+V = %.2f GB)" % (attn_bytes(w) / 2 / 1e9)},
+            "stages_ms": {"routing": route_ms, "attention": attn_ms},
+            "tflops_kept_pairs": flop / (ms_step * 1e-3) / 1e12,
+            "roofline": {"bound": "tensor", "kernel": "sparse_attn_fwd_kernel", "achieved": attn_tflops,
+                         "peak": tc_peak, "unit": "TFLOP/s", "frac": attn_tflops / tc_peak,
+                         "peak_kind": f"{peak_kind} bf16 dense (burst)", "traffic": None,
+                         "flop_per_launch": flop},
+            "routing_roofline": {"bound": "hbm", "achieved": rbytes / (route_ms * 1e-3) / 1e9, "peak": hbm_peak,
+                                 "unit": "GB/s", "frac": rbytes / (route_ms * 1e-3) / 1e9 / hbm_peak,
+                                 "bytes_per_layer": rbytes},
+            "gpu_launches": n_launch_per_step * args.steps,
+            "device_flags": flags,
+            "clocks": clk.summary(),
+            "e2e": e2e,
+            "dense": dense,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

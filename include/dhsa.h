@@ -1,0 +1,176 @@
+/*
+ * dhsa.h -- C ABI of the DHSA prefill hot path on NVIDIA B200 (sm_100a).
+ *
+ * Dynamic Hierarchical Sparse Attention ("Long-Context Modeling with Dynamic
+ * Hierarchical Sparse Attention for Memory-Constrained LLM Inference") routes
+ * attention hierarchically: the sequence is cut into variable-length chunks,
+ * each chunk of Q and K is pooled into one length-normalised vector, the
+ * pooled vectors are scored chunk-to-chunk, each query chunk keeps its
+ * diagonal chunk plus the top-k earlier chunks, and the chunk decision is
+ * expanded to a token keep-set that a causal sparse attention kernel reads.
+ * The four calls below are those four stages, in order.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * - All tensor pointers are DEVICE pointers owned by the caller. The library
+ *   never allocates, frees or synchronises; scratch memory is passed in as a
+ *   `workspace` whose size is given by the matching *_workspace_size query.
+ * - Every compute call is asynchronous on `stream` (a cudaStream_t, passed as
+ *   void*; NULL = the legacy default stream). Host-side argument checks run
+ *   before anything is enqueued; a call that returns an error enqueued nothing.
+ * - Tensors are dense and row-major:
+ *     Q   bf16  [B, Hq,  L, head_dim]
+ *     K,V bf16  [B, Hkv, L, head_dim]      (GQA: query head hq reads kv head hq / (Hq/Hkv))
+ *     off int32 [B, Nmax+1]   chunk c of batch b = tokens [off[b][c], off[b][c+1]);
+ *                             off[b][0] = 0, strictly increasing up to
+ *                             off[b][n_chunks[b]] = L, padded with L after.
+ *     n_chunks int32 [B]      1 <= n_chunks[b] <= Nmax.
+ *   One chunk layout per batch element is shared by all heads and by Q/K/V.
+ * - head_dim must be 128 (the pages' kernel contract: "BF16, causal,
+ *   forward-only, head dimension 128", DHSA README, "Installation").
+ * - Return value: a dhsa_status_t. DHSA_ERR_CUDA keeps the CUDA error code
+ *   for dhsa_last_cuda_error(). Device-side failures (a bounded wait that
+ *   timed out, an offsets table found inconsistent) set a device status word
+ *   that dhsa_check_device_status() reads; compute calls never trap.
+ * - The library holds no per-call state; calls on different streams may run
+ *   concurrently as long as their buffers do not overlap.
+ */
+#ifndef DHSA_H_
+#define DHSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  DHSA_OK = 0,
+  DHSA_ERR_INVALID_ARG = 1,  /* null pointer, non-positive size, Hq % Hkv != 0, k < 0, Nmax > L, ... */
+  DHSA_ERR_UNSUPPORTED = 2,  /* head_dim != 128, or the current device is not sm_100 */
+  DHSA_ERR_CUDA = 3,         /* a CUDA runtime call or launch failed; see dhsa_last_cuda_error() */
+  DHSA_ERR_DEVICE = 4,       /* a kernel reported an error on the device (dhsa_check_device_status) */
+  DHSA_ERR_WORKSPACE = 5     /* workspace pointer null or smaller than the size query asked for */
+} dhsa_status_t;
+
+/* Device status word bits, as returned in *device_flags by dhsa_check_device_status. */
+#define DHSA_DEVFLAG_WAIT_TIMEOUT 0x1  /* a pipeline wait in the attention kernel gave up */
+#define DHSA_DEVFLAG_BAD_OFFSETS 0x2   /* dhsa_validate_offsets found a bad offsets table */
+#define DHSA_DEVFLAG_BAD_SELECTION 0x4 /* the CSR builder met a selected chunk outside [0, i] */
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* dhsa_status_string(int status);
+
+/* CUDA error code (cudaError_t as int) of the last DHSA_ERR_CUDA on this host thread. */
+int dhsa_last_cuda_error(void);
+
+/* ABI version: major * 10000 + minor * 100 + patch. */
+int dhsa_version(void);
+
+/* Synchronises `stream`, reads and clears the current device's status word.
+ * Returns DHSA_ERR_DEVICE if any flag was set (flags returned in
+ * *device_flags when not NULL), DHSA_ERR_CUDA if the stream itself failed. */
+int dhsa_check_device_status(void* stream, uint32_t* device_flags);
+
+/* Checks an offsets table on the device without trusting the host: every
+ * batch element must have 1 <= n_chunks[b] <= Nmax, off[b][0] = 0, strictly
+ * increasing offsets up to off[b][n_chunks[b]] = L and padding equal to L.
+ * A violation sets DHSA_DEVFLAG_BAD_OFFSETS (read it with
+ * dhsa_check_device_status). Asynchronous on `stream`. */
+int dhsa_validate_offsets(const int32_t* off, const int32_t* n_chunks, int B, int Nmax, int L, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * 1. Length-normalised chunk pooling.
+ *    Source: OpenReview abstract (chunk representations aggregate the token
+ *    embeddings of the chunk; the average is scaled by the square root of the
+ *    chunk size) and the gist.science technical summary, "Robust Chunk
+ *    Representation".
+ *
+ *    Xp[b,h,c,:] = (sum over tokens t of chunk c of X[b,h,t,:]) / sqrt(n_c)
+ *
+ *    X   bf16  [B, H, L, head_dim]  (call once with Q, H = Hq; once with K, H = Hkv)
+ *    Xp  fp32  [B, H, Nmax, head_dim], written in full: rows c >= n_chunks[b]
+ *        are set to zero. Sums are accumulated in fp32.
+ * ------------------------------------------------------------------------- */
+int dhsa_chunk_pool(const void* X, int B, int H, int L, int head_dim, const int32_t* off,
+                    const int32_t* n_chunks, int Nmax, float* Xp, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * 2. Chunk similarity and causal per-query-chunk top-k.
+ *    Source: gist.science technical summary, "Hierarchical Routing
+ *    Formulation", Steps 1-2 (a chunk-level similarity matrix; each query
+ *    chunk is routed to a compact set of chunks under the causal constraint).
+ *
+ *    For each row (b, hq, i < n_chunks[b]):
+ *      S[j] = <Qp[b,hq,i,:], Kp[b,hq/G,j,:]> for j < i (fp32 inputs, the dot
+ *             product accumulated in fp64; the diagonal needs no score);
+ *      kept = {i} + the min(k, i) earlier chunks ranked by (S descending,
+ *             j ascending) -- ties go to the lower chunk index;
+ *      sel[b,hq,i, 0 .. n_sel-1] = kept in ascending order (diagonal last),
+ *      the rest of the row = -1; n_sel[b,hq,i] = min(k, i) + 1.
+ *    Rows i >= n_chunks[b] get n_sel = 0 and are filled with -1.
+ *
+ *    Qp fp32 [B, Hq, Nmax, 128], Kp fp32 [B, Hkv, Nmax, 128] (as written by 1.)
+ *    sel   int32 [B, Hq, Nmax, sel_stride], sel_stride = dhsa_sel_stride(k, Nmax)
+ *    n_sel int32 [B, Hq, Nmax]
+ *    k >= Nmax - 1 keeps every earlier chunk (dense causal).
+ *    workspace: dhsa_score_topk_workspace_size(B, Hq, Nmax) bytes (0 when the
+ *    scores of a row block fit in shared memory, i.e. Nmax <= 2048); may be
+ *    NULL when that size is 0.
+ * ------------------------------------------------------------------------- */
+int dhsa_sel_stride(int k, int Nmax);
+size_t dhsa_score_topk_workspace_size(int B, int Hq, int Nmax);
+int dhsa_chunk_score_topk(const float* Qp, const float* Kp, int B, int Hq, int Hkv, int Nmax,
+                          const int32_t* n_chunks, int k, int32_t* sel, int32_t* n_sel, void* workspace,
+                          size_t workspace_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * 3. Upsampling to the token keep-set, stored as a block CSR.
+ *    Source: OpenReview abstract (chunk scores are upsampled to the token
+ *    level to decide which token interactions are kept); gist.science
+ *    technical summary, Step 2 (high-scoring chunks expand into their tokens
+ *    under the causal constraint).
+ *
+ *    Query token t of chunk i keeps key token s iff chunk(s) is in sel(i) and
+ *    s <= t. That set is never materialised: it is the CSR below plus `off`.
+ *    Rows r = (b*Hq + hq)*Nmax + i:
+ *      row_ptr int32 [B*Hq*Nmax + 1]  exclusive prefix sum of n_sel
+ *      col_idx int32 [row_ptr[last]]  kept chunks of row r, ascending (diagonal last)
+ *      cost    int64 [B*Hq*Nmax] or NULL: n_i * sum_{j in sel(i)} n_j, 0 for padded rows
+ *    col_idx needs room for dhsa_csr_nnz_upper(B, Hq, Nmax, k) entries.
+ * ------------------------------------------------------------------------- */
+size_t dhsa_csr_nnz_upper(int B, int Hq, int Nmax, int k);
+int dhsa_build_block_csr(const int32_t* sel, const int32_t* n_sel, int B, int Hq, int Nmax, int k,
+                         const int32_t* off, const int32_t* n_chunks, int32_t* row_ptr, int32_t* col_idx,
+                         int64_t* cost, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * 4. Causal block-sparse attention forward over the kept chunk pairs.
+ *    Source: DHSA README, "Overview" (block-sparse attention extended to
+ *    variable-sized query and key blocks) and "Installation" (BF16, causal,
+ *    forward-only, head dim 128); gist.science technical summary, "Key
+ *    Technical Components" (tiled online-softmax backend that never builds
+ *    the full attention matrix).
+ *
+ *    O[b,hq,t,:] = sum_s softmax_s(scale * <Q[b,hq,t], K[b,hkv,s]>) V[b,hkv,s]
+ *    over the kept keys s of token t only (hkv = hq / (Hq/Hkv)); fp32
+ *    accumulation and softmax statistics, bf16 output (round to nearest).
+ *    Every row of V must be finite, including rows that are not kept (a
+ *    masked key contributes 0 * V[s]).
+ *
+ *    row_ptr / col_idx as written by 3. (cost may be NULL; it is not read yet).
+ *    O bf16 [B, Hq, L, 128]; every token row of every head is written.
+ *    workspace: dhsa_sparse_attn_workspace_size(B, Hq, L, Nmax) bytes.
+ * ------------------------------------------------------------------------- */
+size_t dhsa_sparse_attn_workspace_size(int B, int Hq, int L, int Nmax);
+int dhsa_sparse_attn_fwd(const void* Q, const void* K, const void* V, int B, int Hq, int Hkv, int L,
+                         int head_dim, const int32_t* off, const int32_t* n_chunks, int Nmax,
+                         const int32_t* row_ptr, const int32_t* col_idx, const int64_t* cost,
+                         float softmax_scale, void* O, void* workspace, size_t workspace_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DHSA_H_ */

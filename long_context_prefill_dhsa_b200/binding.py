@@ -1,0 +1,260 @@
+"""ctypes binding of libdhsa (the C ABI in include/dhsa.h).
+
+Argument marshalling only: torch tensors are checked for dtype, shape,
+contiguity and device, then their data pointers and the current CUDA stream
+are handed to the library. Every step of the path runs in the library's CUDA
+kernels; there is no fallback. If the library is missing, loading fails
+loudly (build it with `python -m long_context_prefill_dhsa_b200.build`).
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import re
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libdhsa.so")
+HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "dhsa.h")
+
+DHSA_OK = 0
+STATUS_NAMES = {0: "DHSA_OK", 1: "DHSA_ERR_INVALID_ARG", 2: "DHSA_ERR_UNSUPPORTED", 3: "DHSA_ERR_CUDA",
+                4: "DHSA_ERR_DEVICE", 5: "DHSA_ERR_WORKSPACE"}
+DEVFLAG_WAIT_TIMEOUT, DEVFLAG_BAD_OFFSETS, DEVFLAG_BAD_SELECTION = 0x1, 0x2, 0x4
+
+
+class DHSAError(RuntimeError):
+    def __init__(self, status: int, where: str, cuda_error: int = 0, flags: int = 0):
+        self.status, self.where, self.cuda_error, self.flags = status, where, cuda_error, flags
+        msg = f"{where}: {STATUS_NAMES.get(status, status)}"
+        if cuda_error:
+            msg += f" (cudaError {cuda_error})"
+        if flags:
+            msg += f" (device flags 0x{flags:x})"
+        super().__init__(msg)
+
+
+_c = ctypes
+_P, _I, _F, _SZ = _c.c_void_p, _c.c_int, _c.c_float, _c.c_size_t
+_SIGNATURES = {
+    "dhsa_status_string": (_c.c_char_p, [_I]),
+    "dhsa_last_cuda_error": (_I, []),
+    "dhsa_version": (_I, []),
+    "dhsa_check_device_status": (_I, [_P, _c.POINTER(_c.c_uint32)]),
+    "dhsa_validate_offsets": (_I, [_P, _P, _I, _I, _I, _P]),
+    "dhsa_chunk_pool": (_I, [_P, _I, _I, _I, _I, _P, _P, _I, _P, _P]),
+    "dhsa_sel_stride": (_I, [_I, _I]),
+    "dhsa_score_topk_workspace_size": (_SZ, [_I, _I, _I]),
+    "dhsa_chunk_score_topk": (_I, [_P, _P, _I, _I, _I, _I, _P, _I, _P, _P, _P, _SZ, _P]),
+    "dhsa_csr_nnz_upper": (_SZ, [_I, _I, _I, _I]),
+    "dhsa_build_block_csr": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P]),
+    "dhsa_sparse_attn_workspace_size": (_SZ, [_I, _I, _I, _I]),
+    "dhsa_sparse_attn_fwd": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _I, _P, _P, _P, _F, _P, _P, _SZ, _P]),
+}
+
+_lib: Optional[ctypes.CDLL] = None
+
+
+def load() -> ctypes.CDLL:
+    """Load libdhsa.so (once). Raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m long_context_prefill_dhsa_b200.build`")
+        lib = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGNATURES.items():
+            fn = getattr(lib, name)
+            fn.restype, fn.argtypes = res, args
+        _lib = lib
+    return _lib
+
+
+def header_functions() -> list[str]:
+    """Names of the functions include/dhsa.h declares."""
+    text = open(HEADER_PATH).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(dhsa_[a-z0-9_]+)\s*\(", text)))
+
+
+def _check(status: int, where: str):
+    if status != DHSA_OK:
+        raise DHSAError(status, where, load().dhsa_last_cuda_error() if status == 3 else 0)
+
+
+def _stream_ptr() -> int:
+    return torch.cuda.current_stream().cuda_stream
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else t.data_ptr()
+
+
+def _need(t: torch.Tensor, dtype, shape, name):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name}: expected a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: dtype {t.dtype}, expected {dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name}: must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+# ----------------------------------------------------------------- stage calls
+def check_device_status() -> int:
+    flags = ctypes.c_uint32(0)
+    st = load().dhsa_check_device_status(_stream_ptr(), ctypes.byref(flags))
+    if st != DHSA_OK:
+        raise DHSAError(st, "dhsa_check_device_status", load().dhsa_last_cuda_error() if st == 3 else 0,
+                        flags.value)
+    return flags.value
+
+
+def validate_offsets(off: torch.Tensor, n_chunks: torch.Tensor, L: int):
+    B, n1 = off.shape
+    _need(off, torch.int32, None, "off")
+    _need(n_chunks, torch.int32, (B,), "n_chunks")
+    _check(load().dhsa_validate_offsets(_ptr(off), _ptr(n_chunks), B, n1 - 1, L, _stream_ptr()),
+           "dhsa_validate_offsets")
+
+
+def chunk_pool(X: torch.Tensor, off: torch.Tensor, n_chunks: torch.Tensor, out: Optional[torch.Tensor] = None):
+    """Xp[b,h,c] = sum of chunk c's rows / sqrt(n_c), fp32 [B,H,Nmax,128]."""
+    B, H, L, d = X.shape
+    nmax = off.shape[1] - 1
+    _need(X, torch.bfloat16, None, "X")
+    _need(off, torch.int32, (B, nmax + 1), "off")
+    _need(n_chunks, torch.int32, (B,), "n_chunks")
+    if out is None:
+        out = torch.empty((B, H, nmax, d), dtype=torch.float32, device=X.device)
+    _need(out, torch.float32, (B, H, nmax, d), "out")
+    _check(load().dhsa_chunk_pool(_ptr(X), B, H, L, d, _ptr(off), _ptr(n_chunks), nmax, _ptr(out), _stream_ptr()),
+           "dhsa_chunk_pool")
+    return out
+
+
+def sel_stride(k: int, nmax: int) -> int:
+    return load().dhsa_sel_stride(k, nmax)
+
+
+def chunk_score_topk(Qp: torch.Tensor, Kp: torch.Tensor, n_chunks: torch.Tensor, k: int,
+                     sel: Optional[torch.Tensor] = None, n_sel: Optional[torch.Tensor] = None,
+                     workspace: Optional[torch.Tensor] = None):
+    """sel [B,Hq,Nmax,stride] (ascending, diagonal last, -1 padded) and n_sel [B,Hq,Nmax]."""
+    B, Hq, nmax, d = Qp.shape
+    Hkv = Kp.shape[1]
+    _need(Qp, torch.float32, None, "Qp")
+    _need(Kp, torch.float32, (B, Hkv, nmax, d), "Kp")
+    _need(n_chunks, torch.int32, (B,), "n_chunks")
+    lib = load()
+    stride = lib.dhsa_sel_stride(k, nmax)
+    if sel is None:
+        sel = torch.empty((B, Hq, nmax, stride), dtype=torch.int32, device=Qp.device)
+    if n_sel is None:
+        n_sel = torch.empty((B, Hq, nmax), dtype=torch.int32, device=Qp.device)
+    _need(sel, torch.int32, (B, Hq, nmax, stride), "sel")
+    _need(n_sel, torch.int32, (B, Hq, nmax), "n_sel")
+    ws_bytes = lib.dhsa_score_topk_workspace_size(B, Hq, nmax)
+    if ws_bytes and workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=Qp.device)
+    ws_ptr = _ptr(workspace) if ws_bytes else None
+    ws_len = workspace.numel() * workspace.element_size() if (ws_bytes and workspace is not None) else 0
+    _check(lib.dhsa_chunk_score_topk(_ptr(Qp), _ptr(Kp), B, Hq, Hkv, nmax, _ptr(n_chunks), k, _ptr(sel),
+                                     _ptr(n_sel), ws_ptr, ws_len, _stream_ptr()), "dhsa_chunk_score_topk")
+    return sel, n_sel
+
+
+def build_block_csr(sel: torch.Tensor, n_sel: torch.Tensor, k: int, off: torch.Tensor, n_chunks: torch.Tensor,
+                    row_ptr=None, col_idx=None, cost=None, want_cost: bool = True):
+    B, Hq, nmax, stride = sel.shape
+    lib = load()
+    _need(sel, torch.int32, None, "sel")
+    _need(n_sel, torch.int32, (B, Hq, nmax), "n_sel")
+    if row_ptr is None:
+        row_ptr = torch.empty(B * Hq * nmax + 1, dtype=torch.int32, device=sel.device)
+    if col_idx is None:
+        col_idx = torch.empty(lib.dhsa_csr_nnz_upper(B, Hq, nmax, k), dtype=torch.int32, device=sel.device)
+    if cost is None and want_cost:
+        cost = torch.empty(B * Hq * nmax, dtype=torch.int64, device=sel.device)
+    _check(lib.dhsa_build_block_csr(_ptr(sel), _ptr(n_sel), B, Hq, nmax, k, _ptr(off), _ptr(n_chunks),
+                                    _ptr(row_ptr), _ptr(col_idx), _ptr(cost), _stream_ptr()),
+           "dhsa_build_block_csr")
+    return row_ptr, col_idx, cost
+
+
+def sparse_attn_fwd(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, off: torch.Tensor, n_chunks: torch.Tensor,
+                    row_ptr: torch.Tensor, col_idx: torch.Tensor, cost: Optional[torch.Tensor] = None,
+                    softmax_scale: Optional[float] = None, out: Optional[torch.Tensor] = None,
+                    workspace: Optional[torch.Tensor] = None):
+    B, Hq, L, d = Q.shape
+    Hkv = K.shape[1]
+    nmax = off.shape[1] - 1
+    _need(Q, torch.bfloat16, None, "Q")
+    _need(K, torch.bfloat16, (B, Hkv, L, d), "K")
+    _need(V, torch.bfloat16, (B, Hkv, L, d), "V")
+    lib = load()
+    if out is None:
+        out = torch.empty_like(Q)
+    _need(out, torch.bfloat16, (B, Hq, L, d), "out")
+    ws_bytes = lib.dhsa_sparse_attn_workspace_size(B, Hq, L, nmax)
+    if workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=Q.device)
+    scale = 1.0 / math.sqrt(d) if softmax_scale is None else float(softmax_scale)
+    _check(lib.dhsa_sparse_attn_fwd(_ptr(Q), _ptr(K), _ptr(V), B, Hq, Hkv, L, d, _ptr(off), _ptr(n_chunks), nmax,
+                                    _ptr(row_ptr), _ptr(col_idx), _ptr(cost), scale, _ptr(out), _ptr(workspace),
+                                    workspace.numel(), _stream_ptr()), "dhsa_sparse_attn_fwd")
+    return out
+
+
+# ----------------------------------------------------------------- whole layer
+class DHSAPrefill:
+    """The five calls of one DHSA prefill layer with buffers allocated once.
+
+    run(Q, K, V) does pool(Q), pool(K), score + top-k, CSR build and sparse
+    attention on the current stream and returns O (bf16, like Q).
+    """
+
+    def __init__(self, B: int, Hq: int, Hkv: int, L: int, off: torch.Tensor, n_chunks: torch.Tensor, k: int,
+                 device="cuda", softmax_scale: Optional[float] = None):
+        lib = load()
+        self.B, self.Hq, self.Hkv, self.L, self.k = B, Hq, Hkv, L, k
+        self.off, self.n_chunks = off, n_chunks
+        self.nmax = off.shape[1] - 1
+        nmax = self.nmax
+        dev = torch.device(device)
+        self.scale = 1.0 / math.sqrt(128) if softmax_scale is None else softmax_scale
+        self.Qp = torch.empty((B, Hq, nmax, 128), dtype=torch.float32, device=dev)
+        self.Kp = torch.empty((B, Hkv, nmax, 128), dtype=torch.float32, device=dev)
+        self.stride = lib.dhsa_sel_stride(k, nmax)
+        self.sel = torch.empty((B, Hq, nmax, self.stride), dtype=torch.int32, device=dev)
+        self.n_sel = torch.empty((B, Hq, nmax), dtype=torch.int32, device=dev)
+        ws1 = lib.dhsa_score_topk_workspace_size(B, Hq, nmax)
+        self.ws_topk = torch.empty(max(ws1, 1), dtype=torch.uint8, device=dev) if ws1 else None
+        self.row_ptr = torch.empty(B * Hq * nmax + 1, dtype=torch.int32, device=dev)
+        self.col_idx = torch.empty(lib.dhsa_csr_nnz_upper(B, Hq, nmax, k), dtype=torch.int32, device=dev)
+        self.cost = torch.empty(B * Hq * nmax, dtype=torch.int64, device=dev)
+        self.ws_attn = torch.empty(lib.dhsa_sparse_attn_workspace_size(B, Hq, L, nmax), dtype=torch.uint8,
+                                   device=dev)
+        self.O = torch.empty((B, Hq, L, 128), dtype=torch.bfloat16, device=dev)
+
+    def routing(self, Q, K):
+        chunk_pool(Q, self.off, self.n_chunks, out=self.Qp)
+        chunk_pool(K, self.off, self.n_chunks, out=self.Kp)
+        chunk_score_topk(self.Qp, self.Kp, self.n_chunks, self.k, sel=self.sel, n_sel=self.n_sel,
+                         workspace=self.ws_topk)
+        build_block_csr(self.sel, self.n_sel, self.k, self.off, self.n_chunks, row_ptr=self.row_ptr,
+                        col_idx=self.col_idx, cost=self.cost)
+
+    def attention(self, Q, K, V):
+        return sparse_attn_fwd(Q, K, V, self.off, self.n_chunks, self.row_ptr, self.col_idx, self.cost,
+                               self.scale, out=self.O, workspace=self.ws_attn)
+
+    def run(self, Q, K, V):
+        self.routing(Q, K)
+        return self.attention(Q, K, V)

@@ -1,0 +1,112 @@
+// Length-normalised chunk pooling (stage 1 of the DHSA routing).
+//
+// OpenReview abstract of "Long-Context Modeling with Dynamic Hierarchical
+// Sparse Attention": each chunk is represented by the average of its token
+// embeddings scaled by the square root of the chunk size, i.e.
+//   Xp[b,h,c,:] = sum_{t in chunk c} X[b,h,t,:] / sqrt(n_c).
+//
+// HBM-bound streaming read of X. One warp owns one (b, h, chunk): lanes 0-15
+// read the even rows and lanes 16-31 the odd rows of the chunk, each lane
+// 16 bytes (8 bf16) of the 256-byte row, so a warp instruction moves two full
+// rows; eight rows per lane are in flight per iteration. The two half-warp
+// partial sums are combined with one shuffle, and the 1/sqrt(n) scale is
+// applied on the way out. Warps of one block cover consecutive chunks of the
+// same head, so a block reads a contiguous span of X.
+#include "common.cuh"
+
+namespace dhsa {
+namespace {
+
+__device__ __forceinline__ void add_bf16x8(float (&acc)[8], const uint4& v) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    acc[2 * q] += __uint_as_float(w[q] << 16);
+    acc[2 * q + 1] += __uint_as_float(w[q] & 0xFFFF0000u);
+  }
+}
+
+__global__ void __launch_bounds__(256) chunk_pool_kernel(const uint4* __restrict__ X, int H, int L,
+                                                         const int32_t* __restrict__ off,
+                                                         const int32_t* __restrict__ n_chunks, int Nmax,
+                                                         long long n_rows, float* __restrict__ Xp) {
+  const long long warp = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (warp >= n_rows) return;
+  const int c = (int)(warp % Nmax);
+  const long long bh = warp / Nmax;
+  const int b = (int)(bh / H);
+  const int half = lane >> 4, sub = lane & 15;
+
+  float acc[8];
+#pragma unroll
+  for (int q = 0; q < 8; ++q) acc[q] = 0.f;
+
+  const int n = n_chunks[b];
+  if (c < n) {
+    const int s = off[(long long)b * (Nmax + 1) + c];
+    const int e = off[(long long)b * (Nmax + 1) + c + 1];
+    // row r of head bh starts at uint4 index (bh*L + r) * 16
+    const uint4* head = X + (bh * L) * 16 + sub;
+    int r = s + half;
+    for (; r + 14 < e; r += 16) {
+      uint4 v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[u] = __ldg(head + (long long)(r + 2 * u) * 16);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) add_bf16x8(acc, v[u]);
+    }
+    for (; r < e; r += 2) add_bf16x8(acc, __ldg(head + (long long)r * 16));
+#pragma unroll
+    for (int q = 0; q < 8; ++q) acc[q] += __shfl_xor_sync(0xffffffffu, acc[q], 16);
+    const float root = __fsqrt_rn((float)(e - s));
+#pragma unroll
+    for (int q = 0; q < 8; ++q) acc[q] = __fdiv_rn(acc[q], root);
+  }
+  if (half == 0) {
+    float4* dst = reinterpret_cast<float4*>(Xp + warp * kHeadDim + 8 * sub);
+    dst[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+    dst[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+  }
+}
+
+__global__ void validate_offsets_kernel(const int32_t* __restrict__ off, const int32_t* __restrict__ n_chunks,
+                                        int B, int Nmax, int L, unsigned int* status) {
+  const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= (long long)B * (Nmax + 1)) return;
+  const int b = (int)(idx / (Nmax + 1));
+  const int c = (int)(idx % (Nmax + 1));
+  const int n = n_chunks[b];
+  const int32_t* ob = off + (long long)b * (Nmax + 1);
+  bool bad = (n < 1 || n > Nmax);
+  if (!bad) {
+    if (c == 0) bad = ob[0] != 0;
+    else if (c < n) bad = !(ob[c] > ob[c - 1] && ob[c] < L);
+    else if (c == n) bad = !(ob[c] == L && ob[c] > ob[c - 1]);
+    else bad = ob[c] != L;
+  }
+  if (bad) raise_device_flag(status, DHSA_DEVFLAG_BAD_OFFSETS);
+}
+
+}  // namespace
+
+int launch_chunk_pool(const void* X, int B, int H, int L, const int32_t* off, const int32_t* n_chunks, int Nmax,
+                      float* Xp, cudaStream_t stream) {
+  const long long n_rows = (long long)B * H * Nmax;
+  const int threads = 256;
+  const long long blocks = (n_rows * 32 + threads - 1) / threads;
+  chunk_pool_kernel<<<(unsigned)blocks, threads, 0, stream>>>(static_cast<const uint4*>(X), H, L, off, n_chunks,
+                                                               Nmax, n_rows, Xp);
+  return launch_status();
+}
+
+int launch_validate_offsets(const int32_t* off, const int32_t* n_chunks, int B, int Nmax, int L,
+                            unsigned int* status, cudaStream_t stream) {
+  const long long n = (long long)B * (Nmax + 1);
+  const int threads = 256;
+  validate_offsets_kernel<<<(unsigned)((n + threads - 1) / threads), threads, 0, stream>>>(off, n_chunks, B, Nmax,
+                                                                                            L, status);
+  return launch_status();
+}
+
+}  // namespace dhsa

@@ -1,0 +1,67 @@
+"""The C-ABI library builds, loads and exports every function include/dhsa.h
+declares; host-side argument checks answer without touching a GPU."""
+import ctypes
+
+import pytest
+
+from long_context_prefill_dhsa_b200 import binding, build
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return binding.load()
+
+
+def test_exports_every_declared_function(lib):
+    names = binding.header_functions()
+    assert len(names) >= 13
+    missing = [n for n in names if not hasattr(lib, n)]
+    assert not missing, missing
+    assert set(names) >= set(binding._SIGNATURES)
+
+
+def test_status_strings_and_version(lib):
+    assert lib.dhsa_version() >= 100
+    for code, name in binding.STATUS_NAMES.items():
+        assert lib.dhsa_status_string(code).decode() == name
+    assert lib.dhsa_status_string(99).decode() == "DHSA_ERR_UNKNOWN"
+
+
+def test_size_queries(lib):
+    assert lib.dhsa_sel_stride(8, 55) == 9
+    assert lib.dhsa_sel_stride(100, 55) == 55        # k >= Nmax - 1: every earlier chunk
+    assert lib.dhsa_sel_stride(-1, 55) == 0
+    assert lib.dhsa_csr_nnz_upper(2, 4, 10, 3) == 2 * 4 * 10 * 4
+    assert lib.dhsa_score_topk_workspace_size(1, 32, 823) == 0     # scores fit in shared memory
+    assert lib.dhsa_score_topk_workspace_size(1, 32, 4096) > 0
+    assert lib.dhsa_sparse_attn_workspace_size(1, 32, 131072, 823) >= 16 * 32 * (823 + 1024)
+
+
+FAKE = 1 << 20   # a non-null, 16-byte aligned stand-in pointer; never dereferenced
+
+
+def test_invalid_arguments_rejected_on_host(lib):
+    INV, UNS, WS = 1, 2, 5
+    # pool: null input, bad sizes, head_dim != 128
+    assert lib.dhsa_chunk_pool(None, 1, 1, 8, 128, FAKE, FAKE, 1, FAKE, None) == INV
+    assert lib.dhsa_chunk_pool(FAKE, 0, 1, 8, 128, FAKE, FAKE, 1, FAKE, None) == INV
+    assert lib.dhsa_chunk_pool(FAKE, 1, 1, 8, 128, FAKE, FAKE, 9, FAKE, None) == INV   # Nmax > L
+    assert lib.dhsa_chunk_pool(FAKE + 4, 1, 1, 8, 128, FAKE, FAKE, 1, FAKE, None) == INV  # misaligned
+    assert lib.dhsa_chunk_pool(FAKE, 1, 1, 8, 64, FAKE, FAKE, 1, FAKE, None) == UNS
+    # score/top-k: k < 0, Hq % Hkv != 0, missing workspace for a large Nmax
+    assert lib.dhsa_chunk_score_topk(FAKE, FAKE, 1, 4, 2, 8, FAKE, -1, FAKE, FAKE, None, 0, None) == INV
+    assert lib.dhsa_chunk_score_topk(FAKE, FAKE, 1, 3, 2, 8, FAKE, 1, FAKE, FAKE, None, 0, None) == INV
+    assert lib.dhsa_chunk_score_topk(FAKE, FAKE, 1, 4, 2, 5000, FAKE, 1, FAKE, FAKE, None, 0, None) == WS
+    # CSR: null output
+    assert lib.dhsa_build_block_csr(FAKE, FAKE, 1, 1, 4, 1, FAKE, FAKE, None, FAKE, None, None) == INV
+    # attention: head_dim, scale, workspace
+    args = [FAKE, FAKE, FAKE, 1, 2, 1, 256, 128, FAKE, FAKE, 4, FAKE, FAKE, None]
+    big = lib.dhsa_sparse_attn_workspace_size(1, 2, 256, 4)
+    assert lib.dhsa_sparse_attn_fwd(*args, ctypes.c_float(0.1), FAKE, FAKE, big - 16, None) == WS
+    assert lib.dhsa_sparse_attn_fwd(*args, ctypes.c_float(-1.0), FAKE, FAKE, big, None) == INV
+    args[7] = 96
+    assert lib.dhsa_sparse_attn_fwd(*args, ctypes.c_float(0.1), FAKE, FAKE, big, None) == UNS
+    args[7] = 128
+    args[5] = 3      # Hq % Hkv != 0
+    assert lib.dhsa_sparse_attn_fwd(*args, ctypes.c_float(0.1), FAKE, FAKE, big, None) == INV
