@@ -40,7 +40,8 @@ __device__ __forceinline__ unsigned lanemask_lt() {
 }
 
 // Top-m of keys(buf[0..n)) under (key desc, index asc), written ascending to out.
-// Returns the number written (= m). hist: 256 ints of this warp's shared memory.
+// Requires 0 < m < n. Returns the number written (= m); never writes past
+// out[m-1]. hist: 256 ints of this warp's shared memory.
 __device__ int warp_select_topm(const double* buf, int n, int m, int* hist, int32_t* out) {
   const int lane = threadIdx.x & 31;
   const unsigned full = 0xffffffffu;
@@ -102,10 +103,11 @@ __device__ int warp_select_topm(const double* buf, int n, int m, int* hist, int3
     const bool take = gt || (eq && (eq_seen + __popc(beq & lanemask_lt())) < need);
     eq_seen += __popc(beq);
     const unsigned bt = __ballot_sync(full, take);
-    if (take) out[written + __popc(bt & lanemask_lt())] = j;
+    const int pos = written + __popc(bt & lanemask_lt());
+    if (take && pos < m) out[pos] = j;
     written += __popc(bt);
   }
-  return written;
+  return written < m ? written : m;
 }
 
 __global__ void __launch_bounds__(256) score_topk_kernel(const float* __restrict__ Qp, const float* __restrict__ Kp,
@@ -172,7 +174,7 @@ __global__ void __launch_bounds__(256) score_topk_kernel(const float* __restrict
         if (m == i) {
           for (int j = lane; j < i; j += 32) out[j] = j;
           cnt = i;
-        } else {
+        } else if (m > 0) {
           cnt = warp_select_topm(row_scores, i, m, hist + warp * 256, out);
         }
         if (lane == 0) out[cnt] = i;

@@ -176,9 +176,9 @@ def test_ragged_k_all_sampled_vs_dense(lib):
     """The ragged 64K workload with k = all causal chunks equals dense causal
     attention (sampled query chunks of two heads, checked against the
     oracle's textbook dense attention on the tokens up to each chunk)."""
-    w = I.WORKLOADS["ragged-64k"].with_(k=1 << 20)
+    w = I.WORKLOADS["ragged-64k"]
     d = I.make_inputs(w)
-    _, O = _run_gpu(lib, d, w.k)
+    _, O = _run_gpu(lib, d, 1 << 20)
     off, nc = d["off"], d["n_chunks"]
     rng = np.random.default_rng(11)
     errs = []
