@@ -169,6 +169,38 @@ int dhsa_sparse_attn_fwd(const void* Q, const void* K, const void* V, int B, int
                          const int32_t* row_ptr, const int32_t* col_idx, const int64_t* cost,
                          float softmax_scale, void* O, void* workspace, size_t workspace_bytes, void* stream);
 
+/* ---------------------------------------------------------------------------
+ * 4b. The same attention forward without a caller workspace.
+ *    The paper has no counterpart: this is a deployment variant of 4.
+ *
+ *    For callers that cannot call cudaMalloc: code that runs inside an
+ *    engine's pre-planned device-memory arena (every byte is reserved up
+ *    front, so an extra allocation fails or fragments it), and code on a
+ *    latency-critical path where cudaMalloc's implicit device-wide
+ *    synchronisation would stall other streams. The work list that 4. keeps
+ *    in `workspace` is kept instead in a 4 MiB static device array of the
+ *    library (held by every GPU that loads the library until process exit).
+ *    Problems whose work list does not fit, i.e.
+ *      256 + 16 * B * Hq * (Nmax + ceil(L / 128)) > 4 MiB,
+ *    are rejected with DHSA_ERR_WORKSPACE before anything is enqueued
+ *    (use 4. for those). This call performs no cudaMalloc/cudaFree and calls
+ *    no allocating library routine.
+ *
+ *    The first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress) and caches it; make that first call before any
+ *    stream capture. All calls share the one array and it keeps the last
+ *    call's contents; nothing in it has to start at zero (each call rewrites
+ *    the whole work list and its count). Calls whose executions overlap on
+ *    the GPU (other streams, other host threads) race on the array: order
+ *    them, e.g. on one stream.
+ *
+ *    Arguments, layouts and results are those of dhsa_sparse_attn_fwd.
+ * ------------------------------------------------------------------------- */
+int dhsa_sparse_attn_fwd_noalloc(const void* Q, const void* K, const void* V, int B, int Hq, int Hkv, int L,
+                                 int head_dim, const int32_t* off, const int32_t* n_chunks, int Nmax,
+                                 const int32_t* row_ptr, const int32_t* col_idx, float softmax_scale, void* O,
+                                 void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -53,6 +53,7 @@ _SIGNATURES = {
     "dhsa_build_block_csr": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P]),
     "dhsa_sparse_attn_workspace_size": (_SZ, [_I, _I, _I, _I]),
     "dhsa_sparse_attn_fwd": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _I, _P, _P, _P, _F, _P, _P, _SZ, _P]),
+    "dhsa_sparse_attn_fwd_noalloc": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _I, _P, _P, _F, _P, _P]),
 }
 
 _lib: Optional[ctypes.CDLL] = None
@@ -209,6 +210,28 @@ def sparse_attn_fwd(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, off: torc
     _check(lib.dhsa_sparse_attn_fwd(_ptr(Q), _ptr(K), _ptr(V), B, Hq, Hkv, L, d, _ptr(off), _ptr(n_chunks), nmax,
                                     _ptr(row_ptr), _ptr(col_idx), _ptr(cost), scale, _ptr(out), _ptr(workspace),
                                     workspace.numel(), _stream_ptr()), "dhsa_sparse_attn_fwd")
+    return out
+
+
+def sparse_attn_fwd_noalloc(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, off: torch.Tensor,
+                            n_chunks: torch.Tensor, row_ptr: torch.Tensor, col_idx: torch.Tensor,
+                            softmax_scale: Optional[float] = None, out: Optional[torch.Tensor] = None):
+    """sparse_attn_fwd with the library's static scratch instead of a caller
+    workspace (for callers that cannot allocate; see include/dhsa.h, 4b).
+    `out` should be preallocated by such callers."""
+    B, Hq, L, d = Q.shape
+    Hkv = K.shape[1]
+    nmax = off.shape[1] - 1
+    _need(Q, torch.bfloat16, None, "Q")
+    _need(K, torch.bfloat16, (B, Hkv, L, d), "K")
+    _need(V, torch.bfloat16, (B, Hkv, L, d), "V")
+    if out is None:
+        out = torch.empty_like(Q)
+    _need(out, torch.bfloat16, (B, Hq, L, d), "out")
+    scale = 1.0 / math.sqrt(d) if softmax_scale is None else float(softmax_scale)
+    _check(load().dhsa_sparse_attn_fwd_noalloc(_ptr(Q), _ptr(K), _ptr(V), B, Hq, Hkv, L, d, _ptr(off),
+                                               _ptr(n_chunks), nmax, _ptr(row_ptr), _ptr(col_idx), scale,
+                                               _ptr(out), _stream_ptr()), "dhsa_sparse_attn_fwd_noalloc")
     return out
 
 

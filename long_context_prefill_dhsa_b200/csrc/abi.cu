@@ -22,6 +22,8 @@ int launch_sparse_attn(const void* Q, const void* K, const void* V, int B, int H
                        const int32_t* off, const int32_t* n_chunks, int Nmax, const int32_t* row_ptr,
                        const int32_t* col_idx, float softmax_scale, void* O, void* ws, unsigned int* status,
                        cudaStream_t stream);
+size_t noalloc_scratch_bytes();
+int noalloc_scratch_ptr(void** out);
 
 namespace {
 __device__ unsigned int g_device_status = 0;
@@ -201,6 +203,27 @@ int dhsa_sparse_attn_fwd(const void* Q, const void* K, const void* V, int B, int
   if (!status) return DHSA_ERR_CUDA;
   return launch_sparse_attn(Q, K, V, B, Hq, Hkv, L, off, n_chunks, Nmax, row_ptr, col_idx, softmax_scale, O,
                             workspace, status, static_cast<cudaStream_t>(stream));
+}
+
+int dhsa_sparse_attn_fwd_noalloc(const void* Q, const void* K, const void* V, int B, int Hq, int Hkv, int L,
+                                 int head_dim, const int32_t* off, const int32_t* n_chunks, int Nmax,
+                                 const int32_t* row_ptr, const int32_t* col_idx, float softmax_scale, void* O,
+                                 void* stream) {
+  int st = check_layout(B, Hq, L, Nmax, off, n_chunks);
+  if (st != DHSA_OK) return st;
+  if (!Q || !K || !V || !O || !row_ptr || !col_idx) return DHSA_ERR_INVALID_ARG;
+  if (Hkv <= 0 || Hq % Hkv != 0) return DHSA_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O)) return DHSA_ERR_INVALID_ARG;
+  if (!(softmax_scale > 0.f) || softmax_scale != softmax_scale) return DHSA_ERR_INVALID_ARG;
+  if (head_dim != kHeadDim) return DHSA_ERR_UNSUPPORTED;
+  if (attn_ws_bytes(B, Hq, L, Nmax) > noalloc_scratch_bytes()) return DHSA_ERR_WORKSPACE;
+  if ((st = check_device_sm100()) != DHSA_OK) return st;
+  unsigned int* status = device_status_ptr();
+  if (!status) return DHSA_ERR_CUDA;
+  void* scratch = nullptr;
+  if ((st = noalloc_scratch_ptr(&scratch)) != DHSA_OK) return st;
+  return launch_sparse_attn(Q, K, V, B, Hq, Hkv, L, off, n_chunks, Nmax, row_ptr, col_idx, softmax_scale, O,
+                            scratch, status, static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

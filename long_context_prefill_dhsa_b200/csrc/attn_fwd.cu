@@ -577,6 +577,20 @@ bool make_map(EncodeTiledFn enc, CUtensorMap* m, const void* base, long long row
 
 }  // namespace
 
+// ----------------------------------------------------------- no-allocation variant
+// Scratch for callers that must not allocate device memory. It lives in a
+// file-scope device array that every GPU loading the library holds until the
+// process exits. It backs the same work list the caller's workspace would
+// hold, so the maximum problem is the one whose work list fits:
+// 256 + 16 * B * Hq * (Nmax + ceil(L / 128)) bytes <= 4 MiB.
+constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+constexpr int kNoAllocMaxDevices = 64;
+void* g_noalloc_ptr[kNoAllocMaxDevices] = {nullptr};
+}  // namespace
+
 size_t attn_items_cap(int B, int Hq, int L, int Nmax) {
   return (size_t)B * Hq * ((size_t)Nmax + (size_t)(L + BM - 1) / BM);
 }
@@ -629,6 +643,30 @@ int launch_sparse_attn(const void* Q, const void* K, const void* V, int B, int H
   const int grid = (int)(cap < sms ? cap : sms);
   sparse_attn_fwd_kernel<<<grid, kThreads, kSmemAlloc, stream>>>(maps, prm);
   return launch_status();
+}
+
+}  // namespace dhsa
+
+namespace dhsa {
+
+size_t noalloc_scratch_bytes() { return kNoAllocScratchBytes; }
+
+// Device address of the static scratch on the current device. The host-side
+// name g_noalloc_scratch is only a stand-in, so the address is looked up once
+// per device (on that device's first call) and cached.
+int noalloc_scratch_ptr(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_status(e);
+  if (dev < 0 || dev >= kNoAllocMaxDevices) return DHSA_ERR_UNSUPPORTED;
+  if (!g_noalloc_ptr[dev]) {
+    void* ptr = nullptr;
+    e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_status(e);
+    g_noalloc_ptr[dev] = ptr;
+  }
+  *out = g_noalloc_ptr[dev];
+  return DHSA_OK;
 }
 
 }  // namespace dhsa

@@ -1,0 +1,73 @@
+"""The attention entry point that allocates nothing (dhsa_sparse_attn_fwd_noalloc).
+
+It exists for callers that cannot call cudaMalloc -- code running inside an
+engine's pre-planned device-memory arena, or on a latency-critical path where
+cudaMalloc's implicit device-wide synchronisation would stall other streams.
+Instead of a caller workspace it uses a 4 MiB static device array of the
+library. This file checks, through the C ABI, that its output matches the
+workspace entry point's on two calls in a row (two different problems, so the
+second call runs over the first one's leftover scratch contents), and that a
+problem too large for the static scratch is refused before anything runs.
+It is collected last, and passes alone or after the other tests.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+from long_context_prefill_dhsa_b200 import inputs as I
+from tests import _parity as P
+
+pytestmark = pytest.mark.gpu
+
+needs_gpu = pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")
+
+
+def _routing(binding, w):
+    d = I.make_inputs(w)
+    t = P.to_dev(d)
+    layer = binding.DHSAPrefill(w.B, w.Hq, w.Hkv, w.L, t["off"], t["n_chunks"], w.k)
+    layer.routing(t["Q"], t["K"])
+    return t, layer
+
+
+@needs_gpu
+def test_noalloc_matches_workspace_entry_on_two_calls():
+    from long_context_prefill_dhsa_b200 import binding
+    problems = [I.custom(B=2, Hq=8, Hkv=2, L=3000, lo=1, hi=400, kind="geometric", mean=60.0, k=5, wid=301),
+                I.custom(B=1, Hq=4, Hkv=1, L=1200, lo=20, hi=200, k=3, wid=302)]
+    for w in problems:
+        t, layer = _routing(binding, w)
+        ref = binding.sparse_attn_fwd(t["Q"], t["K"], t["V"], t["off"], t["n_chunks"], layer.row_ptr,
+                                      layer.col_idx)
+        out = torch.full_like(ref, float("nan"))
+        binding.sparse_attn_fwd_noalloc(t["Q"], t["K"], t["V"], t["off"], t["n_chunks"], layer.row_ptr,
+                                        layer.col_idx, out=out)
+        torch.cuda.synchronize()
+        assert binding.check_device_status() == 0
+        err = (out.float() - ref.float()).abs()
+        assert torch.isfinite(out.float()).all()
+        assert err.max().item() <= P.MAX_ABS and err.mean().item() <= P.MEAN_ABS
+        # and against the oracle on a few query chunks, so both are right
+        from oracle import dhsa as ora
+        d = I.make_inputs(w)
+        sel = P.gpu_sel_rows(layer.sel, layer.n_sel)
+        off, nc = d["off"], d["n_chunks"]
+        for i in (0, int(nc[0]) // 2, int(nc[0]) - 1):
+            s, e = int(off[0, i]), int(off[0, i + 1])
+            o_ref = ora.attn_chunk(ora.bf16_to_f64(d["Q"][0, 0]), ora.bf16_to_f64(d["K"][0, 0]),
+                                   ora.bf16_to_f64(d["V"][0, 0]), off[0], sel[0][0][i], i, P.scale())
+            assert np.abs(out[0, 0, s:e].float().cpu().numpy() - o_ref).max() <= P.MAX_ABS
+
+
+@needs_gpu
+def test_noalloc_rejects_problems_beyond_static_scratch():
+    from long_context_prefill_dhsa_b200 import binding
+    lib = binding.load()
+    # 256 + 16 * B*Hq*(Nmax + ceil(L/128)) > 4 MiB for this shape; refused on the host
+    B, Hq, Hkv, L, nmax = 1, 64, 8, 131072, 4096
+    fake = ctypes.c_void_p(1 << 20)
+    st = lib.dhsa_sparse_attn_fwd_noalloc(fake, fake, fake, B, Hq, Hkv, L, 128, fake, fake, nmax, fake, fake,
+                                          ctypes.c_float(0.088), fake, None)
+    assert st == 5   # DHSA_ERR_WORKSPACE
