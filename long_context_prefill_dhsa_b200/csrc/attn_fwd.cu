@@ -16,18 +16,26 @@
 //   into 128-slot key tiles. Each chunk starts on an 8-slot boundary (one
 //   128-byte-swizzle atom = 8 rows x 128 B, so every TMA destination is
 //   1024-byte aligned) and is fetched with TMA boxes of 64/32/16/8 rows at
-//   arbitrary row coordinates. Padding slots and causally hidden keys are
-//   masked in registers through a per-tile slot -> token table.
-// * Warp roles (192 threads): warp 0 = TMA producer (Q tile, K/V ring of
-//   2 stages), warp 1 = tcgen05 MMA issuer (one thread), warps 2-5 = softmax
-//   and epilogue (thread = query row = TMEM lane).
+//   arbitrary row coordinates.
+// * Masking: padding slots are removed inside the tensor core. Every QK^T
+//   gets one extra K=16 MMA step, ones-column x per-slot bias (0 for a kept
+//   key, -inf for a padding slot), so S already holds -inf there. Only tiles
+//   that hold keys of the diagonal chunk past the tile's first query row run
+//   a per-element causal compare (slot token <= query token).
+// * Warp roles (256 threads): warp 0 = TMA producer, warp 1 = tcgen05 MMA
+//   issuer (one thread), warp 2 = scheduler (resolves each work item's chunk
+//   list into a shared-memory ring up to 4 items ahead), warp 3 idle,
+//   warps 4-7 = softmax + epilogue (thread = query row = TMEM lane).
+// * Pipelines: Q double-buffered; separate K and V rings of 2 stages; a K
+//   stage is released as soon as its QK^T completes, a V stage after its PV.
 // * TMEM (512 columns): S double buffer (2 x 128 fp32 columns) and the O
-//   accumulator (128 columns). P = softmax numerators is written back as bf16
-//   into the S buffer it came from and consumed from TMEM by the PV MMA
-//   (A operand in TMEM, V as an N-major shared-memory operand).
+//   accumulator (128 columns). P (bf16) is written back into the S buffer it
+//   came from and consumed from TMEM by the PV MMA (A in TMEM, V as an
+//   N-major shared-memory operand).
 // * Online softmax in the log2 domain; the running max is only raised (and O
 //   rescaled in TMEM) when it grows by more than 8 (a factor 256), which keeps
-//   the final O / l exact while skipping most rescales.
+//   O / l exact while skipping nearly all rescales; only then does the softmax
+//   wait for the previous PV.
 // * Every mbarrier wait is bounded; a timeout sets DHSA_DEVFLAG_WAIT_TIMEOUT,
 //   the CTA drains its own in-flight copies and MMAs (again bounded), frees
 //   its TMEM and exits.
@@ -43,13 +51,19 @@ using namespace ptx;
 
 constexpr int BM = 128;              // query rows per tile
 constexpr int BN = 128;              // key slots per tile
-constexpr int NS = 2;                // K/V pipeline stages
-constexpr int kThreads = 192;
+constexpr int NSK = 2;               // K pipeline stages
+constexpr int NSV = 2;               // V pipeline stages
+constexpr int NTOK = 4;              // slot-token table ring (causal tiles)
+constexpr int NSLOT = 4;             // scheduled work items in flight
+constexpr int SEG_CAP = 64;          // chunk descriptors kept in shared memory per item
+constexpr int kThreads = 256;
 constexpr uint32_t kHalfBytes = 128 * 128;   // 128 rows x 64 bf16 (one 128B-swizzled half tile)
 constexpr uint32_t kTileBytes = 2 * kHalfBytes;
+constexpr uint32_t kBiasBytes = 128 * 16 * 2;  // 128 rows x 16 bf16, no swizzle
 constexpr uint32_t kTmemCols = 512;
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s per wait
 constexpr int kNoToken = 0x7fffffff;
+constexpr uint16_t kBf16One = 0x3F80, kBf16NegInf = 0xFF80;
 
 struct AttnMaps {
   CUtensorMap q;      // box 64 x 128 rows
@@ -69,30 +83,63 @@ struct AttnParams {
   unsigned int* status;
 };
 
+// One scheduled work item, written by the scheduler warp.
 struct ItemMeta {
-  int q0;       // first query token of the tile
-  int q_rows;   // valid query rows (1..128)
-  int T;        // key tiles
-  int pad;
-  long long o_row0;  // global row (in O) of token 0 of this (b, hq)
+  int q0;        // token of the first query row
+  int q_rows;    // valid query rows (1..128)
+  int T;         // key tiles
+  int nseg;      // kept chunks (the last one is the diagonal chunk)
+  int kv_row0;   // global K/V row of token 0 of this (b, kv head)
+  int q_row0;    // global Q/O row of token 0 of this (b, q head)
+  int rp0;       // first CSR entry of the row
+  int b;
+  int i;         // query chunk
+  int c_start;   // first token of chunk i
+  int pad[2];
+};
+struct ItemSlot {
+  ItemMeta m;
+  int2 seg[SEG_CAP];   // (first token, visible length) of the first SEG_CAP kept chunks
 };
 
 // shared-memory layout (offsets from a 1024-aligned base)
 constexpr uint32_t OFF_Q = 0;                                   // 2 x 32 KB
-constexpr uint32_t OFF_K = OFF_Q + 2 * kTileBytes;              // NS x 32 KB
-constexpr uint32_t OFF_V = OFF_K + NS * kTileBytes;             // NS x 32 KB
-constexpr uint32_t OFF_TOK = OFF_V + NS * kTileBytes;           // NS x 128 int
-constexpr uint32_t OFF_FLAG = OFF_TOK + NS * BN * 4;            // NS int
-constexpr uint32_t OFF_META = OFF_FLAG + 16;                    // 2 x ItemMeta
-constexpr uint32_t OFF_BAR = OFF_META + 2 * sizeof(ItemMeta);   // barriers (8 B each)
+constexpr uint32_t OFF_K = OFF_Q + 2 * kTileBytes;              // NSK x 32 KB
+constexpr uint32_t OFF_V = OFF_K + NSK * kTileBytes;            // NSV x 32 KB
+constexpr uint32_t OFF_ONES = OFF_V + NSV * kTileBytes;         // 4 KB
+constexpr uint32_t OFF_BIAS = OFF_ONES + kBiasBytes;            // NSK x 4 KB
+constexpr uint32_t OFF_TOK = OFF_BIAS + NSK * kBiasBytes;       // NTOK x 128 int
+constexpr uint32_t OFF_FLAG = OFF_TOK + NTOK * BN * 4;          // NTOK int
+constexpr uint32_t OFF_SLOT = OFF_FLAG + 16 * ((NTOK * 4 + 15) / 16);
+constexpr uint32_t OFF_BAR = OFF_SLOT + NSLOT * sizeof(ItemSlot);
 enum {
-  B_QFULL = 0, B_QEMPTY = 2, B_IFULL = 4, B_IEMPTY = 6, B_KFULL = 8, B_VFULL = 8 + NS, B_KVEMPTY = 8 + 2 * NS,
-  B_SFULL = 8 + 3 * NS, B_PREADY = 10 + 3 * NS, B_ODONE = 12 + 3 * NS, B_FINAL = 13 + 3 * NS, B_COUNT = 14 + 3 * NS
+  B_QFULL = 0,
+  B_QEMPTY = B_QFULL + 2,
+  B_SLFULL = B_QEMPTY + 2,
+  B_SLEMPTY = B_SLFULL + NSLOT,
+  B_KFULL = B_SLEMPTY + NSLOT,
+  B_KEMPTY = B_KFULL + NSK,
+  B_VFULL = B_KEMPTY + NSK,
+  B_VEMPTY = B_VFULL + NSV,
+  B_TOKFULL = B_VEMPTY + NSV,
+  B_TOKEMPTY = B_TOKFULL + NTOK,
+  B_SFULL = B_TOKEMPTY + NTOK,
+  B_PREADY = B_SFULL + 2,
+  B_ODONE = B_PREADY + 2,
+  B_OFINAL = B_ODONE + 1,
+  B_FINAL = B_OFINAL + 1,
+  B_COUNT = B_FINAL + 1
 };
 constexpr uint32_t OFF_TMEMPTR = OFF_BAR + 8 * B_COUNT;
 constexpr uint32_t OFF_ABORT = OFF_TMEMPTR + 4;
 constexpr uint32_t kSmemBytes = OFF_ABORT + 4;
 constexpr uint32_t kSmemAlloc = kSmemBytes + 1024;  // slack for aligning the base
+static_assert(kSmemAlloc <= 227 * 1024, "shared memory budget");
+static_assert(OFF_BAR % 8 == 0 && OFF_SLOT % 16 == 0, "alignment");
+
+// role warps
+constexpr int W_PRODUCER = 0, W_MMA = 1, W_SCHED = 2, W_SOFTMAX0 = 4;
+constexpr int kSlotConsumers = 1 + 1 + 4;  // producer, MMA thread, 4 softmax warps
 
 __device__ __forceinline__ int round8(int x) { return (x + 7) & ~7; }
 
@@ -105,6 +152,11 @@ __device__ __forceinline__ float fast_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// byte offset of element (row, k) in a 128 x 16 bf16 K-major block without swizzle
+__device__ __forceinline__ uint32_t noswz_off(int row, int k) {
+  return (uint32_t)((row >> 3) * 256 + (k >> 3) * 128 + (row & 7) * 16 + (k & 7) * 2);
 }
 
 struct Flags {
@@ -126,7 +178,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_fwd_kernel(const __gr
   const uint32_t sbase = smem_u32(smem);
   int* slot_tok = reinterpret_cast<int*>(smem + OFF_TOK);
   int* tile_flag = reinterpret_cast<int*>(smem + OFF_FLAG);
-  ItemMeta* meta = reinterpret_cast<ItemMeta*>(smem + OFF_META);
+  ItemSlot* slots = reinterpret_cast<ItemSlot*>(smem + OFF_SLOT);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_ABORT);
   auto bar = [&](int idx) { return sbase + OFF_BAR + 8u * idx; };
 
@@ -134,23 +186,33 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_fwd_kernel(const __gr
   const int n_items = *p.n_items;
 
   // ---------------------------------------------------------------- setup
-  if (warp == 0) {
+  if (warp == W_PRODUCER) {
     if (lane == 0) {
       *abort_flag = 0;
       for (int s = 0; s < 2; ++s) {
         mbar_init(bar(B_QFULL + s), 1);
         mbar_init(bar(B_QEMPTY + s), 1);
-        mbar_init(bar(B_IFULL + s), 1);
-        mbar_init(bar(B_IEMPTY + s), 5);   // MMA thread + 4 softmax warps
         mbar_init(bar(B_SFULL + s), 1);
-        mbar_init(bar(B_PREADY + s), 4);   // 4 softmax warps
+        mbar_init(bar(B_PREADY + s), 4);
       }
-      for (int s = 0; s < NS; ++s) {
+      for (int s = 0; s < NSLOT; ++s) {
+        mbar_init(bar(B_SLFULL + s), 1);
+        mbar_init(bar(B_SLEMPTY + s), kSlotConsumers);
+      }
+      for (int s = 0; s < NSK; ++s) {
         mbar_init(bar(B_KFULL + s), 1);
+        mbar_init(bar(B_KEMPTY + s), 1);
+      }
+      for (int s = 0; s < NSV; ++s) {
         mbar_init(bar(B_VFULL + s), 1);
-        mbar_init(bar(B_KVEMPTY + s), 1);
+        mbar_init(bar(B_VEMPTY + s), 1);
+      }
+      for (int s = 0; s < NTOK; ++s) {
+        mbar_init(bar(B_TOKFULL + s), 1);
+        mbar_init(bar(B_TOKEMPTY + s), 4);
       }
       mbar_init(bar(B_ODONE), 1);
+      mbar_init(bar(B_OFINAL), 1);
       mbar_init(bar(B_FINAL), 1);
       fence_mbar_init();
       prefetch_tmap(&maps.q);
@@ -159,14 +221,18 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_fwd_kernel(const __gr
         prefetch_tmap(&maps.v[s]);
       }
     }
-  } else if (warp == 1) {
+  } else if (warp == W_MMA) {
     tmem_alloc(sbase + OFF_TMEMPTR, kTmemCols);
     tmem_relinquish();
   }
-  // V slots that no TMA ever fills must hold finite values (a masked key
-  // contributes P = 0 times its V row); zero both V stages once.
-  for (uint32_t o = threadIdx.x * 16; o < NS * kTileBytes; o += kThreads * 16)
-    *reinterpret_cast<uint4*>(smem + OFF_V + o) = make_uint4(0, 0, 0, 0);
+  // Slots that no TMA fills in a tile must hold finite values (their logits
+  // get -inf added; a masked V row is multiplied by P = 0): zero every K and
+  // V stage and the bias blocks once; then write the ones column of the bias
+  // step's A operand.
+  for (uint32_t o = threadIdx.x * 16; o < OFF_TOK - OFF_K; o += kThreads * 16)
+    *reinterpret_cast<uint4*>(smem + OFF_K + o) = make_uint4(0, 0, 0, 0);
+  __syncthreads();
+  if (threadIdx.x < BM) *reinterpret_cast<uint16_t*>(smem + OFF_ONES + noswz_off(threadIdx.x, 0)) = kBf16One;
   fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
@@ -174,178 +240,219 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_fwd_kernel(const __gr
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + OFF_TMEMPTR);
   Flags fl{abort_flag, p.status};
 
-  if (warp == 0) {
-    // ============================================================ producer
-    uint32_t g = 0;  // global key-tile counter of this CTA
+  if (warp == W_SCHED) {
+    // ============================================================ scheduler
     int n_local = 0;
-    for (int it = blockIdx.x; it < n_items && !*abort_flag; it += gridDim.x, ++n_local) {
+    for (int it = blockIdx.x; it < n_items; it += gridDim.x, ++n_local) {
+      const int sl = n_local % NSLOT;
+      if (n_local >= NSLOT && !fl.wait(bar(B_SLEMPTY + sl), ((n_local / NSLOT) - 1) & 1)) break;
       const int4 wi = p.items[it];
       const int b = wi.x, hq = wi.y, i = wi.z, tq = wi.w;
       const int32_t* ob = p.off + (long long)b * (p.Nmax + 1);
       const int c_start = ob[i], c_end = ob[i + 1];
       const int q0 = c_start + BM * tq;
       const int q_rows = min(BM, c_end - q0);
-      const int q_last = q0 + q_rows - 1;
       const long long r = ((long long)b * p.Hq + hq) * p.Nmax + i;
       const int rp0 = p.row_ptr[r], rp1 = p.row_ptr[r + 1];
-      const long long kv_row0 = ((long long)b * p.Hkv + hq / p.G) * p.L;
-      const long long q_row0 = ((long long)b * p.Hq + hq) * p.L;
-
-      // first batch of chunk descriptors in lanes, and the total slot count
-      int cj = -1, cst = 0, clen = 0, slots = 0;
+      ItemSlot& S = slots[sl];
+      int nslots = 0;
       for (int q = rp0 + lane; q < rp1; q += 32) {
         const int j = p.col_idx[q];
         const int s0 = ob[j];
-        const int len = (j == i) ? (q_last + 1 - c_start) : (ob[j + 1] - s0);
-        slots += round8(len);
-        if (q < rp0 + 32) { cj = j; cst = s0; clen = len; }
+        const int len = (j == i) ? (q0 + q_rows - c_start) : (ob[j + 1] - s0);
+        nslots += round8(len);
+        if (q - rp0 < SEG_CAP) S.seg[q - rp0] = make_int2(s0, len);
       }
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) slots += __shfl_xor_sync(0xffffffffu, slots, o);
-      const int T = (slots + BN - 1) / BN;
-
-      const int ms = n_local & 1;
-      if (n_local >= 2 && !fl.wait(bar(B_IEMPTY + ms), ((n_local >> 1) - 1) & 1)) break;
+      for (int o = 16; o > 0; o >>= 1) nslots += __shfl_xor_sync(0xffffffffu, nslots, o);
       if (lane == 0) {
-        meta[ms].q0 = q0;
-        meta[ms].q_rows = q_rows;
-        meta[ms].T = T;
-        meta[ms].o_row0 = q_row0;
-        mbar_arrive(bar(B_IFULL + ms));
+        S.m.q0 = q0;
+        S.m.q_rows = q_rows;
+        S.m.T = (nslots + BN - 1) / BN;
+        S.m.nseg = rp1 - rp0;
+        S.m.kv_row0 = (int)(((long long)b * p.Hkv + hq / p.G) * p.L);
+        S.m.q_row0 = (int)(((long long)b * p.Hq + hq) * p.L);
+        S.m.rp0 = rp0;
+        S.m.b = b;
+        S.m.i = i;
+        S.m.c_start = c_start;
       }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(B_SLFULL + sl));
+    }
+  } else if (warp == W_PRODUCER) {
+    // ============================================================ producer
+    uint32_t g = 0;  // global key-tile counter of this CTA
+    int n_local = 0;
+    for (int it = blockIdx.x; it < n_items; it += gridDim.x, ++n_local) {
+      const int sl = n_local % NSLOT;
+      if (!fl.wait(bar(B_SLFULL + sl), (n_local / NSLOT) & 1)) break;
+      const ItemMeta M = slots[sl].m;
+      const int2* seg_s = slots[sl].seg;
+      const int ms = n_local & 1;
       if (n_local >= 2 && !fl.wait(bar(B_QEMPTY + ms), ((n_local >> 1) - 1) & 1)) break;
       if (lane == 0) {
         mbar_arrive_expect_tx(bar(B_QFULL + ms), kTileBytes);
         const uint32_t dq = sbase + OFF_Q + ms * kTileBytes;
-        tma_load_2d(dq, &maps.q, bar(B_QFULL + ms), 0, (int)(q_row0 + q0));
-        tma_load_2d(dq + kHalfBytes, &maps.q, bar(B_QFULL + ms), 64, (int)(q_row0 + q0));
+        tma_load_2d(dq, &maps.q, bar(B_QFULL + ms), 0, M.q_row0 + M.q0);
+        tma_load_2d(dq + kHalfBytes, &maps.q, bar(B_QFULL + ms), 64, M.q_row0 + M.q0);
       }
-
-      int seg_q = rp0, cur = 0, seg_pos = 0;
+      const int32_t* ob = p.off + (long long)M.b * (p.Nmax + 1);
+      // chunk descriptors beyond SEG_CAP are read from global memory, 32 at a time
+      int gbase = -1, g_s0 = 0, g_len = 0;
+      auto desc = [&](int sq) -> int2 {
+        if (sq < SEG_CAP) return seg_s[sq];
+        const int base = sq & ~31;
+        if (base != gbase) {
+          gbase = base;
+          const int q = base + lane;
+          if (q < M.nseg) {
+            const int j = p.col_idx[M.rp0 + q];
+            g_s0 = ob[j];
+            g_len = (j == M.i) ? (M.q0 + M.q_rows - M.c_start) : (ob[j + 1] - g_s0);
+          }
+        }
+        return make_int2(__shfl_sync(0xffffffffu, g_s0, sq & 31), __shfl_sync(0xffffffffu, g_len, sq & 31));
+      };
+      int sq = 0, seg_pos = 0;
       bool ok = true;
-      for (int kt = 0; kt < T; ++kt, ++g) {
-        const int st = g % NS;
-        if (g >= NS && !fl.wait(bar(B_KVEMPTY + st), ((g / NS) - 1) & 1)) { ok = false; break; }
-        int slot = 0, needs_mask = 0;
-        int* tok = slot_tok + st * BN;
-        const uint32_t dk = sbase + OFF_K + st * kTileBytes;
-        const uint32_t dv = sbase + OFF_V + st * kTileBytes;
-        while (slot < BN && seg_q < rp1) {
-          const int j = __shfl_sync(0xffffffffu, cj, cur);
-          const int s0 = __shfl_sync(0xffffffffu, cst, cur);
-          const int len = __shfl_sync(0xffffffffu, clen, cur);
-          const int rows = min(len - seg_pos, BN - slot);
+      for (int kt = 0; kt < M.T; ++kt, ++g) {
+        const int stk = g % NSK, stv = g % NSV, tk = g % NTOK;
+        if (g >= NSK && !fl.wait(bar(B_KEMPTY + stk), ((g / NSK) - 1) & 1)) { ok = false; break; }
+        if (g >= NTOK && !fl.wait(bar(B_TOKEMPTY + tk), ((g / NTOK) - 1) & 1)) { ok = false; break; }
+        int* tok = slot_tok + tk * BN;
+        unsigned char* bias = smem + OFF_BIAS + stk * kBiasBytes;
+        // walk the key stream: lane b holds the b-th TMA box of this tile
+        int slot = 0, causal = 0, nbox = 0, my_y = 0, my_so = 0, my_bx = 0;
+        uint32_t bytes = 0;
+        while (slot < BN && sq < M.nseg) {
+          const int2 dsc = desc(sq);
+          const int rows = min(dsc.y - seg_pos, BN - slot);
           const int groups = (rows + 7) >> 3;
-          const int tok0 = s0 + seg_pos;
-          for (int s = lane; s < groups * 8; s += 32) tok[slot + s] = (s < rows) ? tok0 + s : kNoToken;
-          if (rows < groups * 8 || j == i) needs_mask = 1;
-          if (lane == 0) {
-            int gq = 0;
-            while (gq < groups) {
-              const int rem = groups - gq;
-              const int bx = rem >= 8 ? 3 : rem >= 4 ? 2 : rem >= 2 ? 1 : 0;
-              const int nrows = 8 << bx;
-              const uint32_t bytes = nrows * 128u;
-              const int y = (int)(kv_row0 + tok0 + 8 * gq);
-              const uint32_t so = (uint32_t)(slot + 8 * gq) * 128u;
-              mbar_expect_tx(bar(B_KFULL + st), 2 * bytes);
-              tma_load_2d(dk + so, &maps.k[bx], bar(B_KFULL + st), 0, y);
-              tma_load_2d(dk + kHalfBytes + so, &maps.k[bx], bar(B_KFULL + st), 64, y);
-              mbar_expect_tx(bar(B_VFULL + st), 2 * bytes);
-              tma_load_2d(dv + so, &maps.v[bx], bar(B_VFULL + st), 0, y);
-              tma_load_2d(dv + kHalfBytes + so, &maps.v[bx], bar(B_VFULL + st), 64, y);
-              gq += nrows >> 3;
+          const int tok0 = dsc.x + seg_pos;
+          for (int s = lane; s < groups * 8; s += 32) {
+            const bool valid = s < rows;
+            tok[slot + s] = valid ? tok0 + s : kNoToken;
+            *reinterpret_cast<uint16_t*>(bias + noswz_off(slot + s, 0)) = valid ? 0 : kBf16NegInf;
+          }
+          if (sq == M.nseg - 1 && tok0 + rows - 1 > M.q0) causal = 1;  // diagonal keys past the first query
+          int gq = 0;
+          while (gq < groups) {
+            const int rem = groups - gq;
+            const int bx = rem >= 8 ? 3 : rem >= 4 ? 2 : rem >= 2 ? 1 : 0;
+            if (lane == nbox) {
+              my_y = M.kv_row0 + tok0 + 8 * gq;
+              my_so = (slot + 8 * gq) * 128;
+              my_bx = bx;
             }
+            bytes += (8u << bx) * 256u;
+            ++nbox;
+            gq += 1 << bx;
           }
           slot += groups * 8;
           seg_pos += rows;
-          if (seg_pos == len) {
+          if (seg_pos == dsc.y) {
             seg_pos = 0;
-            ++seg_q;
-            if (++cur == 32 && seg_q < rp1) {
-              cur = 0;
-              const int q = seg_q + lane;
-              if (q < rp1) {
-                const int jj = p.col_idx[q];
-                cj = jj;
-                cst = ob[jj];
-                clen = (jj == i) ? (q_last + 1 - c_start) : (ob[jj + 1] - cst);
-              }
-            }
+            ++sq;
           }
         }
-        for (int s = slot + lane; s < BN; s += 32) tok[s] = kNoToken;
-        if (slot < BN) needs_mask = 1;
-        if (lane == 0) tile_flag[st] = needs_mask;
+        for (int s = slot + lane; s < BN; s += 32) {
+          tok[s] = kNoToken;
+          *reinterpret_cast<uint16_t*>(bias + noswz_off(s, 0)) = kBf16NegInf;
+        }
+        if (lane == 0) tile_flag[tk] = causal;
+        fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-          mbar_arrive(bar(B_KFULL + st));
-          mbar_arrive(bar(B_VFULL + st));
+          mbar_arrive(bar(B_TOKFULL + tk));
+          mbar_arrive_expect_tx(bar(B_KFULL + stk), bytes);
+        }
+        __syncwarp();
+        const uint32_t dk = sbase + OFF_K + stk * kTileBytes;
+        if (lane < nbox) {
+          tma_load_2d(dk + my_so, &maps.k[my_bx], bar(B_KFULL + stk), 0, my_y);
+          tma_load_2d(dk + kHalfBytes + my_so, &maps.k[my_bx], bar(B_KFULL + stk), 64, my_y);
+        }
+        if (g >= NSV && !fl.wait(bar(B_VEMPTY + stv), ((g / NSV) - 1) & 1)) { ok = false; ++g; break; }
+        if (lane == 0) mbar_arrive_expect_tx(bar(B_VFULL + stv), bytes);
+        __syncwarp();
+        const uint32_t dv = sbase + OFF_V + stv * kTileBytes;
+        if (lane < nbox) {
+          tma_load_2d(dv + my_so, &maps.v[my_bx], bar(B_VFULL + stv), 0, my_y);
+          tma_load_2d(dv + kHalfBytes + my_so, &maps.v[my_bx], bar(B_VFULL + stv), 64, my_y);
         }
       }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(B_SLEMPTY + sl));
       if (!ok) break;
     }
     // drain: every copy this warp issued must have landed before teardown
     if (lane == 0) {
-      for (uint32_t gg = (g > NS ? g - NS : 0); gg < g; ++gg) {
-        const int st = gg % NS;
-        mbar_wait(bar(B_KFULL + st), (gg / NS) & 1, kWaitLimitNs);
-        mbar_wait(bar(B_VFULL + st), (gg / NS) & 1, kWaitLimitNs);
-      }
+      for (uint32_t gg = (g > NSK ? g - NSK : 0); gg < g; ++gg)
+        mbar_wait(bar(B_KFULL + gg % NSK), (gg / NSK) & 1, kWaitLimitNs);
+      for (uint32_t gg = (g > NSV ? g - NSV : 0); gg < g; ++gg)
+        mbar_wait(bar(B_VFULL + gg % NSV), (gg / NSV) & 1, kWaitLimitNs);
       for (int n = (n_local > 2 ? n_local - 2 : 0); n < n_local; ++n)
         mbar_wait(bar(B_QFULL + (n & 1)), (n >> 1) & 1, kWaitLimitNs);
     }
-  } else if (warp == 1) {
+  } else if (warp == W_MMA) {
     // ============================================================ MMA issuer
     if (lane == 0) {
       const uint32_t idesc_qk = idesc_bf16_f32(BM, BN, false);
       const uint32_t idesc_pv = idesc_bf16_f32(BM, 128, true);
       const uint32_t tS0 = tmem, tO = tmem + 256;
+      const uint64_t ones_desc = smem_desc_noswz(sbase + OFF_ONES, 128, 256);
       uint32_t g = 0;
       int n_local = 0;
-      auto issue_pv = [&](uint32_t u, bool first) -> bool {
-        const int st = u % NS, sb = u & 1;
+      auto issue_pv = [&](uint32_t u, bool first, bool last) -> bool {
+        const int stv = u % NSV, sb = u & 1;
         if (!fl.wait(bar(B_PREADY + sb), (u >> 1) & 1)) return false;
-        if (!fl.wait(bar(B_VFULL + st), (u / NS) & 1)) return false;
+        if (!fl.wait(bar(B_VFULL + stv), (u / NSV) & 1)) return false;
         tc_fence_after();
-        const uint32_t v0 = sbase + OFF_V + st * kTileBytes;
+        const uint32_t v0 = sbase + OFF_V + stv * kTileBytes;
 #pragma unroll
         for (int ks = 0; ks < BN / 16; ++ks) {
           const uint64_t bdesc = smem_desc_sw128(v0 + ks * 2048, kHalfBytes, 1024);
           mma_ts(tO, tS0 + sb * 128 + ks * 8, bdesc, idesc_pv, (!first || ks > 0) ? 1u : 0u);
         }
-        mma_commit(bar(B_KVEMPTY + st));
+        mma_commit(bar(B_VEMPTY + stv));
         mma_commit(bar(B_ODONE));
+        if (last) mma_commit(bar(B_OFINAL));
         return true;
       };
       for (int it = blockIdx.x; it < n_items; it += gridDim.x, ++n_local) {
+        const int sl = n_local % NSLOT;
+        if (!fl.wait(bar(B_SLFULL + sl), (n_local / NSLOT) & 1)) break;
+        const int T = slots[sl].m.T;
+        mbar_arrive(bar(B_SLEMPTY + sl));
         const int ms = n_local & 1;
-        if (!fl.wait(bar(B_IFULL + ms), (n_local >> 1) & 1)) break;
-        const int T = meta[ms].T;
-        mbar_arrive(bar(B_IEMPTY + ms));
         if (!fl.wait(bar(B_QFULL + ms), (n_local >> 1) & 1)) break;
-        const uint32_t q0 = sbase + OFF_Q + ms * kTileBytes;
+        const uint32_t qa = sbase + OFF_Q + ms * kTileBytes;
         bool ok = true;
         for (int kt = 0; kt < T; ++kt, ++g) {
-          const int st = g % NS, sb = g & 1;
-          if (!fl.wait(bar(B_KFULL + st), (g / NS) & 1)) { ok = false; break; }
+          const int stk = g % NSK, sb = g & 1;
+          if (!fl.wait(bar(B_KFULL + stk), (g / NSK) & 1)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t k0 = sbase + OFF_K + st * kTileBytes;
+          const uint32_t k0 = sbase + OFF_K + stk * kTileBytes;
 #pragma unroll
           for (int ks = 0; ks < 8; ++ks) {
             const uint32_t ko = (ks >> 2) * kHalfBytes + (ks & 3) * 32;
-            const uint64_t adesc = smem_desc_sw128(q0 + ko, 16, 1024);
-            const uint64_t bdesc = smem_desc_sw128(k0 + ko, 16, 1024);
-            mma_ss(tS0 + sb * 128, adesc, bdesc, idesc_qk, ks > 0 ? 1u : 0u);
+            mma_ss(tS0 + sb * 128, smem_desc_sw128(qa + ko, 16, 1024), smem_desc_sw128(k0 + ko, 16, 1024),
+                   idesc_qk, ks > 0 ? 1u : 0u);
           }
+          // S += ones x bias: -inf on padding slots
+          mma_ss(tS0 + sb * 128, ones_desc, smem_desc_noswz(sbase + OFF_BIAS + stk * kBiasBytes, 128, 256),
+                 idesc_qk, 1u);
+          mma_commit(bar(B_KEMPTY + stk));
           mma_commit(bar(B_SFULL + sb));
           if (kt == T - 1) mma_commit(bar(B_QEMPTY + ms));
-          if (kt >= 1 && !issue_pv(g - 1, kt == 1)) { ok = false; break; }
+          if (kt >= 1 && !issue_pv(g - 1, kt == 1, false)) { ok = false; break; }
         }
         if (!ok) break;
         if (T == 0) {
           mma_commit(bar(B_QEMPTY + ms));   // an empty key set: nothing to multiply
-        } else if (!issue_pv(g - 1, T == 1)) {
+          mma_commit(bar(B_OFINAL));
+        } else if (!issue_pv(g - 1, T == 1, true)) {
           break;
         }
       }
@@ -353,24 +460,27 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_fwd_kernel(const __gr
       mma_commit(bar(B_FINAL));
       mbar_wait(bar(B_FINAL), 0, kWaitLimitNs);
     }
-  } else {
+  } else if (warp >= W_SOFTMAX0) {
     // ============================================================ softmax + epilogue
     const int quarter = warp & 3;             // TMEM lanes 32*quarter .. +31
     const int row = quarter * 32 + lane;      // query row within the tile
     const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
     const uint32_t tS0 = tmem + lane_addr, tO = tmem + lane_addr + 256;
-    uint32_t g = 0, pv_seen = 0;
+    const float c = p.scale_log2;
+    uint32_t g = 0;
     int n_local = 0;
     for (int it = blockIdx.x; it < n_items; it += gridDim.x, ++n_local) {
-      const int ms = n_local & 1;
-      if (!fl.wait(bar(B_IFULL + ms), (n_local >> 1) & 1)) break;
-      const ItemMeta mt = meta[ms];
-      const int qt = mt.q0 + row;
+      const int sl = n_local % NSLOT;
+      if (!fl.wait(bar(B_SLFULL + sl), (n_local / NSLOT) & 1)) break;
+      const ItemMeta M = slots[sl].m;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(B_SLEMPTY + sl));
+      const int qt = M.q0 + row;
       float m_used = -INFINITY, l_sum = 0.f;
       bool ok = true;
-      for (int kt = 0; kt < mt.T; ++kt, ++g) {
-        const int st = g % NS, sb = g & 1;
-        if (!fl.wait(bar(B_SFULL + sb), (g >> 1) & 1) || !fl.wait(bar(B_KFULL + st), (g / NS) & 1)) {
+      for (int kt = 0; kt < M.T; ++kt, ++g) {
+        const int sb = g & 1, tk = g % NTOK;
+        if (!fl.wait(bar(B_SFULL + sb), (g >> 1) & 1) || !fl.wait(bar(B_TOKFULL + tk), (g / NTOK) & 1)) {
           ok = false;
           break;
         }
@@ -381,63 +491,60 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_fwd_kernel(const __gr
         tmem_ld32(tS0 + sb * 128 + 64, *reinterpret_cast<uint32_t(*)[32]>(s + 64));
         tmem_ld32(tS0 + sb * 128 + 96, *reinterpret_cast<uint32_t(*)[32]>(s + 96));
         tmem_wait_ld();
-        float mx = -INFINITY;
-        if (tile_flag[st]) {
-          const int4* tok4 = reinterpret_cast<const int4*>(slot_tok + st * BN);
+        if (tile_flag[tk]) {
+          const int4* tok4 = reinterpret_cast<const int4*>(slot_tok + tk * BN);
 #pragma unroll
           for (int c4 = 0; c4 < BN / 4; ++c4) {
-            const int4 tk = tok4[c4];
-            const int tks[4] = {tk.x, tk.y, tk.z, tk.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int c = 4 * c4 + e;
-              const float v = (tks[e] <= qt) ? __uint_as_float(s[c]) * p.scale_log2 : -INFINITY;
-              s[c] = __float_as_uint(v);
-              mx = fmaxf(mx, v);
-            }
-          }
-        } else {
-#pragma unroll
-          for (int c = 0; c < BN; ++c) {
-            const float v = __uint_as_float(s[c]) * p.scale_log2;
-            s[c] = __float_as_uint(v);
-            mx = fmaxf(mx, v);
+            const int4 tq = tok4[c4];
+            if (tq.x > qt) s[4 * c4 + 0] = __float_as_uint(-INFINITY);
+            if (tq.y > qt) s[4 * c4 + 1] = __float_as_uint(-INFINITY);
+            if (tq.z > qt) s[4 * c4 + 2] = __float_as_uint(-INFINITY);
+            if (tq.w > qt) s[4 * c4 + 3] = __float_as_uint(-INFINITY);
           }
         }
-        const float m_new = fmaxf(m_used, mx);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(B_TOKEMPTY + tk));
+        // row max over raw scores, 8 independent chains
+        float mx8[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) mx8[e] = __uint_as_float(s[e]);
+#pragma unroll
+        for (int cc = 8; cc < BN; ++cc) mx8[cc & 7] = fmaxf(mx8[cc & 7], __uint_as_float(s[cc]));
+        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+        const float m_new = fmaxf(m_used, mx * c);
         const bool rescale = m_new > m_used + 8.0f;  // also true on the first tile
-        if (kt > 0) {
-          // PV of the previous tile must be complete before O is touched or
-          // its P buffer's neighbour is overwritten
-          if (!fl.wait(bar(B_ODONE), pv_seen & 1)) { ok = false; break; }
-          ++pv_seen;
+        if (kt > 0 && __any_sync(0xffffffffu, rescale)) {
+          // O may only be touched once the previous tile's PV has finished
+          if (!fl.wait(bar(B_ODONE), (g - 1) & 1)) { ok = false; break; }
           tc_fence_after();
-          if (__any_sync(0xffffffffu, rescale)) {
-            const float f = rescale ? fast_exp2(m_used - m_new) : 1.f;
+          const float f = rescale ? fast_exp2(m_used - m_new) : 1.f;
 #pragma unroll
-            for (int c4 = 0; c4 < 4; ++c4) {
-              uint32_t o[32];
-              tmem_ld32(tO + 32 * c4, o);
-              tmem_wait_ld();
+          for (int c4 = 0; c4 < 4; ++c4) {
+            uint32_t o[32];
+            tmem_ld32(tO + 32 * c4, o);
+            tmem_wait_ld();
 #pragma unroll
-              for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
-              tmem_st32(tO + 32 * c4, o);
-            }
-            tmem_wait_st();
-            if (rescale) l_sum *= f;
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
+            tmem_st32(tO + 32 * c4, o);
           }
+          tmem_wait_st();
+          if (rescale) l_sum *= f;
         }
         if (rescale) m_used = m_new;
-        float rs = 0.f;
+        const float neg_m = -m_used;
+        float rs8[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) rs8[e] = 0.f;
         uint32_t pk[BN / 2];
 #pragma unroll
-        for (int c = 0; c < BN / 2; ++c) {
-          const float p0 = fast_exp2(__uint_as_float(s[2 * c]) - m_used);
-          const float p1 = fast_exp2(__uint_as_float(s[2 * c + 1]) - m_used);
-          rs += p0 + p1;
-          pk[c] = pack_bf16x2(p0, p1);
+        for (int cc = 0; cc < BN / 2; ++cc) {
+          const float p0 = fast_exp2(fmaf(__uint_as_float(s[2 * cc]), c, neg_m));
+          const float p1 = fast_exp2(fmaf(__uint_as_float(s[2 * cc + 1]), c, neg_m));
+          rs8[cc & 7] += p0 + p1;
+          pk[cc] = pack_bf16x2(p0, p1);
         }
-        l_sum += rs;
+        l_sum += ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
         tmem_st32(tS0 + sb * 128 + 0, *reinterpret_cast<uint32_t(*)[32]>(pk + 0));
         tmem_st32(tS0 + sb * 128 + 32, *reinterpret_cast<uint32_t(*)[32]>(pk + 32));
         tmem_wait_st();
@@ -448,23 +555,20 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_fwd_kernel(const __gr
       if (!ok) break;
       // epilogue: O / l -> bf16 (an empty key set, which valid CSR input never
       // has, writes zeros)
-      if (mt.T > 0) {
-        if (!fl.wait(bar(B_ODONE), pv_seen & 1)) break;
-        ++pv_seen;
-      }
+      if (!fl.wait(bar(B_OFINAL), n_local & 1)) break;
       tc_fence_after();
-      const float inv_l = mt.T > 0 ? 1.f / l_sum : 0.f;
-      __nv_bfloat16* orow = p.O + (mt.o_row0 + qt) * kHeadDim;
+      const float inv_l = M.T > 0 ? 1.f / l_sum : 0.f;
+      __nv_bfloat16* orow = p.O + ((long long)M.q_row0 + qt) * kHeadDim;
 #pragma unroll
       for (int c4 = 0; c4 < 4; ++c4) {
         uint32_t o[32];
         tmem_ld32(tO + 32 * c4, o);
         tmem_wait_ld();
-        if (mt.T == 0) {
+        if (M.T == 0) {
 #pragma unroll
           for (int e = 0; e < 32; ++e) o[e] = 0u;
         }
-        if (row < mt.q_rows) {
+        if (row < M.q_rows) {
           uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c4);
 #pragma unroll
           for (int v = 0; v < 4; ++v) {
@@ -478,8 +582,6 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_fwd_kernel(const __gr
         }
       }
       tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(B_IEMPTY + ms));
     }
   }
 
@@ -488,7 +590,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_fwd_kernel(const __gr
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem, kTmemCols);
+  if (warp == W_MMA) tmem_dealloc(tmem, kTmemCols);
 }
 
 // Work list: one item per (b, hq, chunk i, 128-row tile of i), ordered
