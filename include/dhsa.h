@@ -103,8 +103,10 @@ int dhsa_chunk_pool(const void* X, int B, int H, int L, int head_dim, const int3
  *    chunk is routed to a compact set of chunks under the causal constraint).
  *
  *    For each row (b, hq, i < n_chunks[b]):
- *      S[j] = <Qp[b,hq,i,:], Kp[b,hq/G,j,:]> for j < i (fp32 inputs, the dot
- *             product accumulated in fp64; the diagonal needs no score);
+ *      S[j] = <Qp[b,hq,i,:], Kp[b,hq/G,j,:]> for j < i, ranked as the fp64
+ *             dot product of the fp32 inputs (computed in fp32; only scores
+ *             within the fp32 rounding bound of the cut are re-scored in
+ *             fp64); the diagonal needs no score;
  *      kept = {i} + the min(k, i) earlier chunks ranked by (S descending,
  *             j ascending) -- ties go to the lower chunk index;
  *      sel[b,hq,i, 0 .. n_sel-1] = kept in ascending order (diagonal last),
@@ -115,9 +117,10 @@ int dhsa_chunk_pool(const void* X, int B, int H, int L, int head_dim, const int3
  *    sel   int32 [B, Hq, Nmax, sel_stride], sel_stride = dhsa_sel_stride(k, Nmax)
  *    n_sel int32 [B, Hq, Nmax]
  *    k >= Nmax - 1 keeps every earlier chunk (dense causal).
- *    workspace: dhsa_score_topk_workspace_size(B, Hq, Nmax) bytes (0 when the
- *    scores of a row block fit in shared memory, i.e. Nmax <= 2048); may be
- *    NULL when that size is 0.
+ *    workspace: dhsa_score_topk_workspace_size(B, Hq, Nmax) bytes: pooled-key
+ *    norms plus the packed fp32 scores (row i keeps its i scores) of a batch
+ *    of heads -- all heads when they fit in 256 MiB, else as many as fit
+ *    (at least one); the call then loops over head batches.
  * ------------------------------------------------------------------------- */
 int dhsa_sel_stride(int k, int Nmax);
 size_t dhsa_score_topk_workspace_size(int B, int Hq, int Nmax);

@@ -7,30 +7,37 @@
 // causal constraint (Step 2). Here: S[i][j] = <Qp_i, Kp_j> for j < i, and the
 // kept set is {i} + the min(k, i) earlier chunks ranked by (S desc, j asc).
 //
-// Layout of the work: one CTA of 8 warps owns 8 consecutive query chunks
-// (rows) of one (b, hq). Scores are exact dot products of the fp32 pooled
-// vectors accumulated in fp64 (fp32 x fp32 products are exact in fp64), so
-// the ranking is decided on values within ~1e-7 relative of the real-number
-// scores. Key tiles of 32 pooled rows are staged in shared memory as fp64;
-// lane l of warp w scores key j0+l against row w. A row's scores stay in
-// shared memory (or, for very many chunks, in a per-CTA workspace slice), and
-// each warp then selects its row's top-k with an 8-pass, 8-bit radix select
-// over an order-preserving 64-bit key, breaking ties at the threshold value
-// by the lowest chunk index. The selected indices come out ascending.
+// The ranking is decided on the fp64 dot products of the fp32 pooled vectors
+// (fp32 x fp32 products are exact in fp64), but only a handful of scores per
+// row are ever computed in fp64:
+//   1. kn kernel: ||Kp_j||_2 for every pooled key row (rounded up).
+//   2. score kernel: fp32 FFMA scores of 64-row x 128-key tiles of the lower
+//      triangle (register-tiled, both operands staged in shared memory),
+//      stored packed per row (row i holds its i scores) in the workspace.
+//   3. select kernel, one warp per row: an 8-bit radix select over the
+//      order-preserving fp32 keys finds the m-th largest fp32 score T. The
+//      fp32 dot product of n = 128 terms is within gamma_n * ||q|| * ||k||
+//      of the exact one (gamma_n = n u / (1 - n u), u = 2^-24), so with D
+//      = 2 gamma_n ||q_i|| max_j ||k_j|| every score above T + D is in the
+//      exact top-m and every score below T - D is out. Only the band
+//      [T - D, T + D] is re-scored in fp64 and ranked exactly (ties to the
+//      lower index). The kept indices are written ascending, diagonal last.
+// For very many chunks the workspace is processed in batches of heads.
 #include "common.cuh"
 
 namespace dhsa {
 namespace {
 
-constexpr int kRows = 8;          // query chunks per CTA (one per warp)
-constexpr int kJT = 32;           // key chunks per staged tile
-constexpr int kKsStride = kHeadDim + 1;
-constexpr int kSmemScoreCap = 2048;  // largest Nmax whose row-block scores stay in shared memory
-constexpr int kWsCtas = 512;      // CTAs of the workspace-backed path
+constexpr int TR = 64;            // query rows per score tile
+constexpr int TK = 128;           // keys per score tile
+constexpr int kKsStride = kHeadDim + 4;
+constexpr size_t kWsCap = size_t(256) << 20;   // scores of one head batch
+constexpr double kU = 5.9604644775390625e-08;   // 2^-24
+constexpr double kGamma = 128.0 * kU / (1.0 - 128.0 * kU);
 
-__device__ __forceinline__ unsigned long long order_key(double s) {
-  const unsigned long long u = (unsigned long long)__double_as_longlong(s);
-  return (u >> 63) ? ~u : (u | 0x8000000000000000ull);
+__device__ __forceinline__ unsigned order_key32(float s) {
+  const unsigned u = __float_as_uint(s);
+  return (u >> 31) ? ~u : (u | 0x80000000u);
 }
 
 __device__ __forceinline__ unsigned lanemask_lt() {
@@ -39,158 +46,322 @@ __device__ __forceinline__ unsigned lanemask_lt() {
   return m;
 }
 
-// Top-m of keys(buf[0..n)) under (key desc, index asc), written ascending to out.
-// Requires 0 < m < n. Returns the number written (= m); never writes past
-// out[m-1]. hist: 256 ints of this warp's shared memory.
-__device__ int warp_select_topm(const double* buf, int n, int m, int* hist, int32_t* out) {
+__host__ __device__ __forceinline__ long long tri(long long i) { return i * (i - 1) / 2; }
+
+// ------------------------------------------------------------------ 1. key norms
+__global__ void __launch_bounds__(256) key_norm_kernel(const float* __restrict__ Kp, long long rows,
+                                                       float* __restrict__ kn) {
+  const long long r = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
-  const unsigned full = 0xffffffffu;
-  unsigned long long prefix = 0, mask = 0;
-  int need = m;
-  for (int shift = 56; shift >= 0; shift -= 8) {
-    for (int q = lane; q < 256; q += 32) hist[q] = 0;
-    __syncwarp();
-    for (int j = lane; j < n; j += 32) {
-      const unsigned long long kk = order_key(buf[j]);
-      if ((kk & mask) == prefix) atomicAdd(&hist[(kk >> shift) & 255], 1);
-    }
-    __syncwarp();
-    int c[8], lsum = 0;
+  if (r >= rows) return;
+  const float4 v = reinterpret_cast<const float4*>(Kp + r * kHeadDim)[lane];
+  double s = (double)v.x * v.x + (double)v.y * v.y + (double)v.z * v.z + (double)v.w * v.w;
 #pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      c[q] = hist[255 - 8 * lane - q];
-      lsum += c[q];
-    }
-    int incl = lsum;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int t = __shfl_up_sync(full, incl, o);
-      if (lane >= o) incl += t;
-    }
-    const int excl = incl - lsum;
-    const unsigned ball = __ballot_sync(full, excl < need && need <= incl);
-    const int src = __ffs(ball) - 1;
-    int digit = 0, above = 0;
-    if (lane == src) {
-      int run = excl;
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        if (run + c[q] >= need) {
-          digit = 255 - 8 * lane - q;
-          above = run;
-          break;
-        }
-        run += c[q];
-      }
-    }
-    digit = __shfl_sync(full, digit, src);
-    above = __shfl_sync(full, above, src);
-    prefix |= (unsigned long long)digit << shift;
-    mask |= 0xFFull << shift;
-    need -= above;
-    __syncwarp();
-  }
-  // prefix is now the m-th largest key; take every larger key and the `need`
-  // lowest-index keys equal to it, in ascending index order.
-  int written = 0, eq_seen = 0;
-  for (int j0 = 0; j0 < n; j0 += 32) {
-    const int j = j0 + lane;
-    const bool valid = j < n;
-    const unsigned long long kk = valid ? order_key(buf[j]) : 0ull;
-    const bool gt = valid && kk > prefix;
-    const bool eq = valid && kk == prefix;
-    const unsigned beq = __ballot_sync(full, eq);
-    const bool take = gt || (eq && (eq_seen + __popc(beq & lanemask_lt())) < need);
-    eq_seen += __popc(beq);
-    const unsigned bt = __ballot_sync(full, take);
-    const int pos = written + __popc(bt & lanemask_lt());
-    if (take && pos < m) out[pos] = j;
-    written += __popc(bt);
-  }
-  return written < m ? written : m;
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  if (lane == 0) kn[r] = (float)(sqrt(s) * (1.0 + 1e-6));   // fp32 rounding covered by the margin
 }
 
-__global__ void __launch_bounds__(256) score_topk_kernel(const float* __restrict__ Qp, const float* __restrict__ Kp,
-                                                         int Hq, int G, int Nmax,
-                                                         const int32_t* __restrict__ n_chunks, int k, int stride,
-                                                         int32_t* __restrict__ sel, int32_t* __restrict__ n_sel,
-                                                         long long n_blocks, double* __restrict__ ws) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  double* Qs = reinterpret_cast<double*>(smem_raw);                 // [kRows][128]
-  double* Ks = Qs + kRows * kHeadDim;                               // [kJT][129]
-  int* hist = reinterpret_cast<int*>(Ks + kJT * kKsStride);         // [kRows][256]
-  double* sbuf = ws ? ws + (long long)blockIdx.x * kRows * Nmax
-                    : reinterpret_cast<double*>(hist + kRows * 256);  // [kRows][Nmax]
-
+// ------------------------------------------------------------------ 2. fp32 score tiles
+__global__ void __launch_bounds__(256, 2) score_tile_kernel(const float* __restrict__ Qp,
+                                                         const float* __restrict__ Kp, int Hq, int G, int Nmax,
+                                                         const int32_t* __restrict__ n_chunks, long long bh0,
+                                                         int n_rb, int n_kb, float* __restrict__ ws) {
+  extern __shared__ __align__(16) float sm[];
+  float* Qs = sm;                        // [TR][128]
+  float* Ks = sm + TR * kHeadDim;        // [TK][132]
+  const int kb = blockIdx.x % n_kb, rb = blockIdx.x / n_kb;
+  const long long bh = bh0 + blockIdx.y;
+  const int b = (int)(bh / Hq), hq = (int)(bh % Hq);
+  const int n = n_chunks[b];
+  const int i0 = rb * TR, j0 = kb * TK;
+  const int i_hi = min(i0 + TR, n);                 // rows [i0, i_hi)
+  if (i0 >= n || j0 >= i_hi - 1) return;            // no j < i in this tile
+  const long long kv_row0 = ((long long)b * (Hq / G) + hq / G) * Nmax;
+  for (int idx = threadIdx.x; idx < TR * 32; idx += blockDim.x) {
+    const int r = idx >> 5, c4 = idx & 31;
+    const int i = i0 + r;
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (i < n) v = reinterpret_cast<const float4*>(Qp + (bh * Nmax + i) * kHeadDim)[c4];
+    reinterpret_cast<float4*>(Qs + r * kHeadDim)[c4] = v;
+  }
+  for (int idx = threadIdx.x; idx < TK * 32; idx += blockDim.x) {
+    const int r = idx >> 5, c4 = idx & 31;
+    const int j = j0 + r;
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (j < n) v = reinterpret_cast<const float4*>(Kp + (kv_row0 + j) * kHeadDim)[c4];
+    reinterpret_cast<float4*>(Ks + r * kKsStride)[c4] = v;
+  }
+  __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int blocks_per_head = (Nmax + kRows - 1) / kRows;
-
-  for (long long blk = blockIdx.x; blk < n_blocks; blk += gridDim.x) {
-    const long long bh = blk / blocks_per_head;             // b * Hq + hq
-    const int i0 = (int)(blk % blocks_per_head) * kRows;
-    const int b = (int)(bh / Hq), hq = (int)(bh % Hq);
-    const int n = n_chunks[b];
-    const long long kv_row0 = ((long long)b * (Hq / G) + hq / G) * Nmax;
-
-    // stage the block's pooled queries as fp64
-    for (int idx = threadIdx.x; idx < kRows * kHeadDim; idx += blockDim.x) {
-      const int r = idx / kHeadDim, d = idx % kHeadDim;
-      const int i = i0 + r;
-      Qs[idx] = (i < n) ? (double)Qp[(bh * Nmax + i) * kHeadDim + d] : 0.0;
-    }
-    const int i_last = min(i0 + kRows, n) - 1;               // largest real row in the block
-    const int i = i0 + warp;
-    double* row_scores = sbuf + warp * Nmax;
-    for (int j0 = 0; j0 < i_last; j0 += kJT) {
-      __syncthreads();
-      for (int idx = threadIdx.x; idx < kJT * kHeadDim; idx += blockDim.x) {
-        const int r = idx / kHeadDim, d = idx % kHeadDim;
-        const int j = j0 + r;
-        Ks[r * kKsStride + d] = (j < n) ? (double)Kp[(kv_row0 + j) * kHeadDim + d] : 0.0;
-      }
-      __syncthreads();
-      const int j = j0 + lane;
-      if (i < n && j < i) {
-        const double* q = Qs + warp * kHeadDim;
-        const double* kr = Ks + lane * kKsStride;
-        double a0 = 0.0, a1 = 0.0, a2 = 0.0, a3 = 0.0;
-#pragma unroll 8
-        for (int d = 0; d < kHeadDim; d += 4) {
-          a0 = fma(q[d], kr[d], a0);
-          a1 = fma(q[d + 1], kr[d + 1], a1);
-          a2 = fma(q[d + 2], kr[d + 2], a2);
-          a3 = fma(q[d + 3], kr[d + 3], a3);
-        }
-        row_scores[j] = (a0 + a1) + (a2 + a3);
+  float acc[8][4];
+#pragma unroll
+  for (int r = 0; r < 8; ++r)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) acc[r][c] = 0.f;
+#pragma unroll 2
+  for (int d = 0; d < kHeadDim; d += 4) {
+    float4 kv[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) kv[c] = *reinterpret_cast<const float4*>(Ks + (lane + 32 * c) * kKsStride + d);
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      const float4 qv = *reinterpret_cast<const float4*>(Qs + (warp * 8 + r) * kHeadDim + d);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        acc[r][c] = fmaf(qv.x, kv[c].x, acc[r][c]);
+        acc[r][c] = fmaf(qv.y, kv[c].y, acc[r][c]);
+        acc[r][c] = fmaf(qv.z, kv[c].z, acc[r][c]);
+        acc[r][c] = fmaf(qv.w, kv[c].w, acc[r][c]);
       }
     }
-    __syncthreads();
-    // selection: warp per row
-    if (i < Nmax) {
-      int32_t* out = sel + (bh * Nmax + i) * stride;
-      int cnt = 0;
-      if (i < n) {
-        const int m = min(k, i);
-        if (m == i) {
-          for (int j = lane; j < i; j += 32) out[j] = j;
-          cnt = i;
-        } else if (m > 0) {
-          cnt = warp_select_topm(row_scores, i, m, hist + warp * 256, out);
-        }
-        if (lane == 0) out[cnt] = i;
-        cnt += 1;
-      }
-      for (int q = cnt + lane; q < stride; q += 32) out[q] = -1;
-      if (lane == 0) n_sel[bh * Nmax + i] = cnt;
+  }
+  float* head = ws + blockIdx.y * tri(Nmax);
+#pragma unroll
+  for (int r = 0; r < 8; ++r) {
+    const int i = i0 + warp * 8 + r;
+    if (i >= i_hi) continue;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const int j = j0 + lane + 32 * c;
+      if (j < i) head[tri(i) + j] = acc[r][c];
     }
-    __syncthreads();
   }
 }
 
-size_t smem_bytes(int Nmax, bool use_ws) {
-  size_t s = sizeof(double) * (kRows * kHeadDim + kJT * kKsStride) + sizeof(int) * kRows * 256;
-  if (!use_ws) s += sizeof(double) * (size_t)kRows * Nmax;
-  return s;
+// ------------------------------------------------------------------ 3. selection
+__device__ double exact_score(const float* __restrict__ q, const float* __restrict__ k) {
+  double a0 = 0.0, a1 = 0.0, a2 = 0.0, a3 = 0.0;
+  for (int d = 0; d < kHeadDim; d += 4) {
+    const float4 x = *reinterpret_cast<const float4*>(q + d);
+    const float4 y = *reinterpret_cast<const float4*>(k + d);
+    a0 = fma((double)x.x, (double)y.x, a0);
+    a1 = fma((double)x.y, (double)y.y, a1);
+    a2 = fma((double)x.z, (double)y.z, a2);
+    a3 = fma((double)x.w, (double)y.w, a3);
+  }
+  return (a0 + a1) + (a2 + a3);
+}
+
+// (score desc, index asc) as one comparison: does (sa, ja) rank above (sb, jb)?
+__device__ __forceinline__ bool ranks_above(double sa, int ja, double sb, int jb) {
+  return sa > sb || (sa == sb && ja < jb);
+}
+
+__global__ void __launch_bounds__(256) select_kernel(const float* __restrict__ Qp, const float* __restrict__ Kp,
+                                                     const float* __restrict__ kn, int Hq, int G, int Nmax,
+                                                     const int32_t* __restrict__ n_chunks, int k, int stride,
+                                                     long long bh0, long long n_rows,
+                                                     const float* __restrict__ ws, int32_t* __restrict__ sel,
+                                                     int32_t* __restrict__ n_sel) {
+  __shared__ int hist_all[8][256];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const unsigned full = 0xffffffffu;
+  const long long wr = (long long)blockIdx.x * 8 + warp;      // row within the head batch
+  if (wr >= n_rows) return;
+  const long long bhl = wr / Nmax;
+  const int i = (int)(wr % Nmax);
+  const long long bh = bh0 + bhl;
+  const int b = (int)(bh / Hq), hq = (int)(bh % Hq);
+  const int n = n_chunks[b];
+  int32_t* out = sel + (bh * Nmax + i) * stride;
+  int* hist = hist_all[warp];
+  int cnt = 0;
+  if (i < n) {
+    const int m = min(k, i);
+    if (m == i) {
+      for (int j = lane; j < i; j += 32) out[j] = j;
+      cnt = i;
+    } else if (m > 0) {
+      const float* row = ws + bhl * tri(Nmax) + tri(i);
+      // --- radix select of the m-th largest fp32 key
+      unsigned prefix = 0, mask = 0;
+      int need = m;
+      for (int shift = 24; shift >= 0; shift -= 8) {
+        for (int q = lane; q < 256; q += 32) hist[q] = 0;
+        __syncwarp();
+        for (int j = lane; j < i; j += 32) {
+          const unsigned kk = order_key32(row[j]);
+          if ((kk & mask) == prefix) atomicAdd(&hist[(kk >> shift) & 255], 1);
+        }
+        __syncwarp();
+        int c[8], lsum = 0;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          c[q] = hist[255 - 8 * lane - q];
+          lsum += c[q];
+        }
+        int incl = lsum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int t = __shfl_up_sync(full, incl, o);
+          if (lane >= o) incl += t;
+        }
+        const int excl = incl - lsum;
+        const unsigned ball = __ballot_sync(full, excl < need && need <= incl);
+        const int src = __ffs(ball) - 1;
+        int digit = 0, above = 0;
+        if (lane == src) {
+          int run = excl;
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            if (run + c[q] >= need) {
+              digit = 255 - 8 * lane - q;
+              above = run;
+              break;
+            }
+            run += c[q];
+          }
+        }
+        digit = __shfl_sync(full, digit, src);
+        above = __shfl_sync(full, above, src);
+        prefix |= (unsigned)digit << shift;
+        mask |= 0xFFu << shift;
+        need -= above;
+        __syncwarp();
+      }
+      const unsigned tu = (prefix & 0x80000000u) ? (prefix & 0x7fffffffu) : ~prefix;
+      const double T = (double)__uint_as_float(tu);
+      // --- rounding band
+      const long long kv_row0 = ((long long)b * (Hq / G) + hq / G) * Nmax;
+      const float* qrow = Qp + (bh * Nmax + i) * kHeadDim;
+      const float4 qv = reinterpret_cast<const float4*>(qrow)[lane];
+      double qq = (double)qv.x * qv.x + (double)qv.y * qv.y + (double)qv.z * qv.z + (double)qv.w * qv.w;
+      float kmax = 0.f;
+      for (int j = lane; j < i; j += 32) kmax = fmaxf(kmax, kn[kv_row0 + j]);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        qq += __shfl_xor_sync(full, qq, o);
+        kmax = fmaxf(kmax, __shfl_xor_sync(full, kmax, o));
+      }
+      const double D = 2.0 * kGamma * sqrt(qq) * (1.0 + 1e-6) * (double)kmax;
+      const double lo = T - D, hi = T + D;
+      int a = 0, nc = 0;
+      for (int j = lane; j < i; j += 32) {
+        const double s = (double)row[j];
+        a += s > hi;
+        nc += (s >= lo && s <= hi);
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        a += __shfl_xor_sync(full, a, o);
+        nc += __shfl_xor_sync(full, nc, o);
+      }
+      const int r = m - a;              // 1 <= r <= nc
+      // --- exact cut (E*, j*) among the band: the r-th by (exact desc, j asc)
+      double cutE = -INFINITY;
+      int cutJ = 0x7fffffff;
+      bool take_all_band = (r >= nc);
+      if (!take_all_band) {
+        if (nc <= 32) {
+          // compact the band into lanes 0..nc-1 (through this warp's free
+          // histogram area), score exactly, bitonic sort best-first
+          int base = 0;
+          for (int j0 = 0; j0 < i; j0 += 32) {
+            const int j = j0 + lane;
+            bool inb = false;
+            if (j < i) {
+              const double s = (double)row[j];
+              inb = s >= lo && s <= hi;
+            }
+            const unsigned bb = __ballot_sync(full, inb);
+            if (inb) hist[base + __popc(bb & lanemask_lt())] = j;
+            base += __popc(bb);
+          }
+          __syncwarp();
+          const int my_j = lane < nc ? hist[lane] : -1;
+          __syncwarp();
+          double my_e = -INFINITY;
+          int my_key_j = 0x7fffffff;
+          if (my_j >= 0) {
+            my_e = exact_score(qrow, Kp + (kv_row0 + my_j) * kHeadDim);
+            my_key_j = my_j;
+          }
+          // bitonic sort of 32 (e, j) pairs, best first
+#pragma unroll
+          for (int size = 2; size <= 32; size <<= 1) {
+#pragma unroll
+            for (int stride2 = size >> 1; stride2 > 0; stride2 >>= 1) {
+              const double oe = __shfl_xor_sync(full, my_e, stride2);
+              const int oj = __shfl_xor_sync(full, my_key_j, stride2);
+              const bool up = ((lane & size) == 0);          // this block sorts best-first
+              const bool lower = ((lane & stride2) == 0);
+              const bool mine_above = ranks_above(my_e, my_key_j, oe, oj);
+              const bool keep_mine = (lower == up) ? mine_above : !mine_above;
+              if (!keep_mine) {
+                my_e = oe;
+                my_key_j = oj;
+              }
+            }
+          }
+          cutE = __shfl_sync(full, my_e, r - 1);
+          cutJ = __shfl_sync(full, my_key_j, r - 1);
+        } else {
+          // many candidates (heavy ties): r rounds of "best below the previous pick"
+          double pe = INFINITY;
+          int pj = -1;
+          for (int t = 0; t < r; ++t) {
+            double be = -INFINITY;
+            int bj = 0x7fffffff;
+            for (int j = lane; j < i; j += 32) {
+              const double s = (double)row[j];
+              if (s < lo || s > hi) continue;
+              const double e = exact_score(qrow, Kp + (kv_row0 + j) * kHeadDim);
+              if (ranks_above(pe, pj, e, j) && ranks_above(e, j, be, bj)) {
+                be = e;
+                bj = j;
+              }
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+              const double oe = __shfl_xor_sync(full, be, o);
+              const int oj = __shfl_xor_sync(full, bj, o);
+              if (ranks_above(oe, oj, be, bj)) {
+                be = oe;
+                bj = oj;
+              }
+            }
+            pe = be;
+            pj = bj;
+          }
+          cutE = pe;
+          cutJ = pj;
+        }
+      }
+      // --- output, ascending
+      int written = 0;
+      for (int j0 = 0; j0 < i; j0 += 32) {
+        const int j = j0 + lane;
+        bool take = false;
+        if (j < i) {
+          const double s = (double)row[j];
+          if (s > hi) {
+            take = true;
+          } else if (s >= lo) {
+            take = take_all_band ||
+                   !ranks_above(cutE, cutJ, exact_score(qrow, Kp + (kv_row0 + j) * kHeadDim), j);
+          }
+        }
+        const unsigned bt = __ballot_sync(full, take);
+        const int pos = written + __popc(bt & lanemask_lt());
+        if (take && pos < m) out[pos] = j;
+        written += __popc(bt);
+      }
+      cnt = written < m ? written : m;
+    }
+    if (lane == 0) out[cnt] = i;
+    cnt += 1;
+  }
+  for (int q = cnt + lane; q < stride; q += 32) out[q] = -1;
+  if (lane == 0) n_sel[bh * Nmax + i] = cnt;
+}
+
+long long heads_per_batch(int B, int Hq, int Nmax) {
+  const size_t per_head = sizeof(float) * (size_t)tri(Nmax);
+  long long h = per_head ? (long long)(kWsCap / per_head) : (long long)B * Hq;
+  if (h < 1) h = 1;
+  if (h > (long long)B * Hq) h = (long long)B * Hq;
+  if (h > 65535) h = 65535;   // grid.y limit
+  return h;
 }
 
 }  // namespace
@@ -198,23 +369,39 @@ size_t smem_bytes(int Nmax, bool use_ws) {
 int score_topk_stride(int k, int Nmax) { return (k < Nmax - 1 ? k : Nmax - 1) + 1; }
 
 size_t score_topk_ws_bytes(int B, int Hq, int Nmax) {
-  if (Nmax <= kSmemScoreCap) return 0;
-  return sizeof(double) * (size_t)kWsCtas * kRows * Nmax;
+  // key norms (B * Hq rows at most, since Hkv <= Hq) + packed scores of one head batch
+  const size_t kn = sizeof(float) * (size_t)B * Hq * Nmax;
+  const size_t scores = sizeof(float) * (size_t)tri(Nmax) * heads_per_batch(B, Hq, Nmax);
+  return 256 + ((kn + 255) & ~size_t(255)) + scores;
 }
 
 int launch_score_topk(const float* Qp, const float* Kp, int B, int Hq, int Hkv, int Nmax, const int32_t* n_chunks,
                       int k, int32_t* sel, int32_t* n_sel, void* ws, cudaStream_t stream) {
-  const bool use_ws = Nmax > kSmemScoreCap;
-  const long long n_blocks = (long long)B * Hq * ((Nmax + kRows - 1) / kRows);
-  const size_t smem = smem_bytes(Nmax, use_ws);
-  cudaError_t e = cudaFuncSetAttribute(score_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  const int G = Hq / Hkv;
+  const int stride = score_topk_stride(k, Nmax);
+  float* kn = reinterpret_cast<float*>(static_cast<char*>(ws) + 256);
+  const size_t kn_bytes = (sizeof(float) * (size_t)B * Hq * Nmax + 255) & ~size_t(255);
+  float* scores = reinterpret_cast<float*>(static_cast<char*>(ws) + 256 + kn_bytes);
+  const long long kv_rows = (long long)B * Hkv * Nmax;
+  key_norm_kernel<<<(unsigned)((kv_rows * 32 + 255) / 256), 256, 0, stream>>>(Kp, kv_rows, kn);
+  int st = launch_status();
+  if (st != DHSA_OK) return st;
+  const size_t smem = sizeof(float) * (TR * kHeadDim + TK * kKsStride);
+  cudaError_t e = cudaFuncSetAttribute(score_tile_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return cuda_status(e);
-  long long grid = use_ws ? (n_blocks < kWsCtas ? n_blocks : kWsCtas) : n_blocks;
-  if (grid > 0x7fffffffLL) grid = 0x7fffffffLL;
-  score_topk_kernel<<<(unsigned)grid, 256, smem, stream>>>(Qp, Kp, Hq, Hq / Hkv, Nmax, n_chunks, k,
-                                                            score_topk_stride(k, Nmax), sel, n_sel, n_blocks,
-                                                            use_ws ? static_cast<double*>(ws) : nullptr);
-  return launch_status();
+  const int n_rb = (Nmax + TR - 1) / TR, n_kb = (Nmax + TK - 1) / TK;
+  const long long total = (long long)B * Hq, hb = heads_per_batch(B, Hq, Nmax);
+  for (long long h0 = 0; h0 < total; h0 += hb) {
+    const long long nh = (total - h0 < hb) ? total - h0 : hb;
+    dim3 grid((unsigned)(n_rb * n_kb), (unsigned)nh);
+    score_tile_kernel<<<grid, 256, smem, stream>>>(Qp, Kp, Hq, G, Nmax, n_chunks, h0, n_rb, n_kb, scores);
+    if ((st = launch_status()) != DHSA_OK) return st;
+    const long long rows = nh * Nmax;
+    select_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(Qp, Kp, kn, Hq, G, Nmax, n_chunks, k, stride, h0,
+                                                                  rows, scores, sel, n_sel);
+    if ((st = launch_status()) != DHSA_OK) return st;
+  }
+  return DHSA_OK;
 }
 
 }  // namespace dhsa

@@ -33,8 +33,11 @@ def test_size_queries(lib):
     assert lib.dhsa_sel_stride(100, 55) == 55        # k >= Nmax - 1: every earlier chunk
     assert lib.dhsa_sel_stride(-1, 55) == 0
     assert lib.dhsa_csr_nnz_upper(2, 4, 10, 3) == 2 * 4 * 10 * 4
-    assert lib.dhsa_score_topk_workspace_size(1, 32, 823) == 0     # scores fit in shared memory
-    assert lib.dhsa_score_topk_workspace_size(1, 32, 4096) > 0
+    # key norms + packed lower-triangle fp32 scores of all heads (they fit in 256 MiB)
+    assert lib.dhsa_score_topk_workspace_size(1, 32, 823) >= 4 * 32 * (823 * 822 // 2 + 823)
+    # very many chunks: one head's scores at a time (the call loops over heads)
+    one_head = 4 * (20000 * 19999 // 2)
+    assert one_head <= lib.dhsa_score_topk_workspace_size(1, 32, 20000) < one_head + (4 << 20)
     assert lib.dhsa_sparse_attn_workspace_size(1, 32, 131072, 823) >= 16 * 32 * (823 + 1024)
 
 
@@ -52,7 +55,8 @@ def test_invalid_arguments_rejected_on_host(lib):
     # score/top-k: k < 0, Hq % Hkv != 0, missing workspace for a large Nmax
     assert lib.dhsa_chunk_score_topk(FAKE, FAKE, 1, 4, 2, 8, FAKE, -1, FAKE, FAKE, None, 0, None) == INV
     assert lib.dhsa_chunk_score_topk(FAKE, FAKE, 1, 3, 2, 8, FAKE, 1, FAKE, FAKE, None, 0, None) == INV
-    assert lib.dhsa_chunk_score_topk(FAKE, FAKE, 1, 4, 2, 5000, FAKE, 1, FAKE, FAKE, None, 0, None) == WS
+    assert lib.dhsa_chunk_score_topk(FAKE, FAKE, 1, 4, 2, 8, FAKE, 1, FAKE, FAKE, None, 0, None) == WS
+    assert lib.dhsa_chunk_score_topk(FAKE, FAKE, 1, 4, 2, 8, FAKE, 1, FAKE, FAKE, FAKE, 64, None) == WS
     # CSR: null output
     assert lib.dhsa_build_block_csr(FAKE, FAKE, 1, 1, 4, 1, FAKE, FAKE, None, FAKE, None, None) == INV
     # attention: head_dim, scale, workspace

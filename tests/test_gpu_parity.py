@@ -101,6 +101,67 @@ def test_k_all_equals_dense(lib):
     assert mx <= P.MAX_ABS and mean <= P.MEAN_ABS
 
 
+def _tie_inputs(kind):
+    """Equal-length chunks whose pooled keys tie exactly: "pairs" copies the K
+    rows of chunk 2c onto chunk 2c+1, "all" gives every key token the same row."""
+    w = I.custom(B=1, Hq=4, Hkv=2, L=16 * 90, lo=16, hi=16, k=7, wid=110 if kind == "pairs" else 111)
+    d = I.make_inputs(w)
+    K = d["K"]
+    if kind == "pairs":
+        for c in range(0, 89, 2):
+            K[:, :, 16 * (c + 1):16 * (c + 2)] = K[:, :, 16 * c:16 * (c + 1)]
+    else:
+        K[:] = K[:, :, :1]
+    return w, d
+
+
+@needs_gpu
+@pytest.mark.parametrize("kind", ["pairs", "all"])
+def test_exact_ties_resolve_to_lower_index(lib, kind):
+    """Exactly tied chunk scores (the degenerate case of the ranking) must be
+    resolved like the oracle: the lower chunk index wins, with no tolerance."""
+    w, d = _tie_inputs(kind)
+    layer, O = _run_gpu(lib, d, w.k)
+    Q, K, V, Qp, Kp, S, sel_ora = P.oracle_full(d, w.k)
+    sel_gpu = P.gpu_sel_rows(layer.sel, layer.n_sel)
+    for h in range(w.Hq):
+        for i in range(int(d["n_chunks"][0])):
+            assert np.array_equal(sel_gpu[0][h][i], sel_ora[0][h][i]), (kind, h, i)
+    if kind == "all":
+        for h in range(w.Hq):
+            for i in range(int(d["n_chunks"][0])):
+                assert list(sel_gpu[0][h][i]) == list(range(min(w.k, i))) + [i]
+    mx, mean = P.compare_out(O, ora.attn_sparse(Q, K, V, d["off"], d["n_chunks"], sel_gpu))
+    assert mx <= P.MAX_ABS and mean <= P.MEAN_ABS
+
+
+@needs_gpu
+def test_many_chunks_head_batched_scores(lib):
+    """~8000 one- or two-token chunks per sequence: the score workspace no
+    longer holds every head at once, so the score/top-k call loops over head
+    batches. Selection is checked row by row against the oracle."""
+    w = I.custom(B=1, Hq=4, Hkv=2, L=12000, lo=1, hi=2, k=12, wid=112)
+    d = I.make_inputs(w)
+    nmax = d["off"].shape[1] - 1
+    assert 4 * nmax * (nmax - 1) // 2 * w.B * w.Hq > (256 << 20)
+    layer, O = _run_gpu(lib, d, w.k)
+    Q, K, V = (ora.bf16_to_f64(d[x]) for x in "QKV")
+    Qp = ora.chunk_pool(Q, d["off"], d["n_chunks"], nmax)
+    Kp = ora.chunk_pool(K, d["off"], d["n_chunks"], nmax)
+    S = ora.chunk_scores(Qp, Kp, d["n_chunks"])
+    sel_ora = ora.select(S, d["n_chunks"], w.k)
+    sel_gpu = P.gpu_sel_rows(layer.sel, layer.n_sel)
+    rows, mism = P.compare_selection(S, sel_ora, sel_gpu, d["n_chunks"], w.k)
+    print(f"many-chunks: rows={rows} near-tie swaps={mism}")
+    rng = np.random.default_rng(3)
+    n = int(d["n_chunks"][0])
+    for i in rng.choice(n, size=40, replace=False):
+        s0, e0 = int(d["off"][0, i]), int(d["off"][0, i + 1])
+        for h in (0, 3):
+            ref = ora.attn_chunk(Q[0, h], K[0, h // 2], V[0, h // 2], d["off"][0], sel_gpu[0][h][i], int(i), P.scale())
+            assert np.abs(O[0, h, s0:e0].float().cpu().numpy() - ref).max() <= P.MAX_ABS
+
+
 @needs_gpu
 def test_two_calls_same_result(lib):
     d = I.make_inputs(SMALL["geometric"])
