@@ -15,8 +15,10 @@
 // * Key stream: the kept chunks of row (b, hq, i) are concatenated and packed
 //   into 128-slot key tiles. Each chunk starts on an 8-slot boundary (one
 //   128-byte-swizzle atom = 8 rows x 128 B, so every TMA destination is
-//   1024-byte aligned) and is fetched with TMA boxes of 64/32/16/8 rows at
-//   arbitrary row coordinates.
+//   1024-byte aligned) and each piece of a chunk inside a tile is fetched with
+//   a single TMA box per head-dim half (16 tensor maps, box heights 8..128
+//   rows) at an arbitrary row coordinate: a TMA op has a fixed cost of tens
+//   of cycles, so splitting pieces into small boxes starves the pipeline.
 // * Masking: padding slots are removed inside the tensor core. Every QK^T
 //   gets one extra K=16 MMA step, ones-column x per-slot bias (0 for a kept
 //   key, -inf for a padding slot), so S already holds -inf there. Only tiles
@@ -67,8 +69,8 @@ constexpr uint16_t kBf16One = 0x3F80, kBf16NegInf = 0xFF80;
 
 struct AttnMaps {
   CUtensorMap q;      // box 64 x 128 rows
-  CUtensorMap k[4];   // boxes 64 x {8,16,32,64} rows
-  CUtensorMap v[4];
+  CUtensorMap k[16];  // boxes 64 cols x 8*(n+1) rows: one TMA per chunk piece and head-dim half
+  CUtensorMap v[16];
 };
 
 struct AttnParams {
@@ -216,7 +218,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_fwd_kernel(const __gr
       mbar_init(bar(B_FINAL), 1);
       fence_mbar_init();
       prefetch_tmap(&maps.q);
-      for (int s = 0; s < 4; ++s) {
+      for (int s = 0; s < 16; ++s) {
         prefetch_tmap(&maps.k[s]);
         prefetch_tmap(&maps.v[s]);
       }
@@ -336,19 +338,15 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_fwd_kernel(const __gr
             *reinterpret_cast<uint16_t*>(bias + noswz_off(slot + s, 0)) = valid ? 0 : kBf16NegInf;
           }
           if (sq == M.nseg - 1 && tok0 + rows - 1 > M.q0) causal = 1;  // diagonal keys past the first query
-          int gq = 0;
-          while (gq < groups) {
-            const int rem = groups - gq;
-            const int bx = rem >= 8 ? 3 : rem >= 4 ? 2 : rem >= 2 ? 1 : 0;
-            if (lane == nbox) {
-              my_y = M.kv_row0 + tok0 + 8 * gq;
-              my_so = (slot + 8 * gq) * 128;
-              my_bx = bx;
-            }
-            bytes += (8u << bx) * 256u;
-            ++nbox;
-            gq += 1 << bx;
+          // the whole piece in one box per head-dim half (per-op TMA cost
+          // dominates for small boxes, so never split a piece)
+          if (lane == nbox) {
+            my_y = M.kv_row0 + tok0;
+            my_so = slot * 128;
+            my_bx = groups - 1;
           }
+          bytes += (uint32_t)groups * 8u * 256u;
+          ++nbox;
           slot += groups * 8;
           seg_pos += rows;
           if (seg_pos == dsc.y) {
@@ -708,9 +706,9 @@ int launch_sparse_attn(const void* Q, const void* K, const void* V, int B, int H
   AttnMaps maps;
   const long long q_rows = (long long)B * Hq * L, kv_rows = (long long)B * Hkv * L;
   bool ok = make_map(enc, &maps.q, Q, q_rows, BM);
-  for (int s = 0; s < 4; ++s) {
-    ok = ok && make_map(enc, &maps.k[s], K, kv_rows, 8 << s);
-    ok = ok && make_map(enc, &maps.v[s], V, kv_rows, 8 << s);
+  for (int s = 0; s < 16; ++s) {
+    ok = ok && make_map(enc, &maps.k[s], K, kv_rows, 8 * (s + 1));
+    ok = ok && make_map(enc, &maps.v[s], V, kv_rows, 8 * (s + 1));
   }
   if (!ok) return DHSA_ERR_INVALID_ARG;
 
