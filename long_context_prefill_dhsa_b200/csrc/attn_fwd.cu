@@ -164,9 +164,10 @@ __device__ __forceinline__ uint32_t noswz_off(int row, int k) {
 struct Flags {
   volatile int* abort;
   unsigned int* status;
-  __device__ bool wait(uint32_t bar, uint32_t parity) {
+  __device__ __forceinline__ bool wait(uint32_t bar, uint32_t parity) {
+    if (mbar_test_wait(bar, parity)) return true;   // fast path: already complete
     if (*abort) return false;
-    if (mbar_wait(bar, parity, kWaitLimitNs)) return true;
+    if (mbar_wait_slow(bar, parity, kWaitLimitNs)) return true;
     *abort = 1;
     raise_device_flag(status, DHSA_DEVFLAG_WAIT_TIMEOUT);
     return false;
