@@ -20,7 +20,6 @@ import json
 import math
 import os
 import statistics
-import subprocess
 import sys
 import threading
 import time
@@ -31,6 +30,13 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "ms per layer (mask+attn) and TFLOP/s on kept pairs at 128K, % of roofline"
+ATTN_SRC = os.path.join(ROOT, "long_context_prefill_dhsa_b200", "csrc", "attn_fwd.cu")
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one attention
+# launch from an ncu capture of the 32K layer, scaled by tokens (x4) to the
+# 128K layer; only valid for the kernel source it was measured on.
+ATTN_TRAFFIC = {"sha256_prefix": "305eaf29c8ca570f",
+                "bytes_per_launch": {"llama3.1-8b-32k": 6.442e8, "llama3.1-8b-128k": 2.577e9},
+                "source": "ncu --set full capture of the 32K layer; 128K scaled x4 by tokens"}
 PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS = 6650.0, 1590.0
 
@@ -47,6 +53,15 @@ def parse():
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     return ap.parse_args()
+
+
+def attn_traffic(workload_name):
+    import hashlib
+    sha = hashlib.sha256(open(ATTN_SRC, "rb").read()).hexdigest()[:16]
+    if sha != ATTN_TRAFFIC["sha256_prefix"]:
+        return None, "kernel changed since the ncu capture"
+    v = ATTN_TRAFFIC["bytes_per_launch"].get(workload_name)
+    return v, ATTN_TRAFFIC["source"] if v is not None else "no capture for this workload"
 
 
 def peaks():
@@ -303,6 +318,7 @@ def main():
     hbm_peak, tc_peak, peak_kind = peaks()
     attn_tflops = flop / (attn_ms * 1e-3) / 1e12
     rbytes = routing_bytes(w, nmax, w.k)
+    traffic, traffic_src = attn_traffic(w.name)
 
     # end to end through the public API with host buffers (pinned), on this rank
     e2e = None
@@ -384,8 +400,8 @@ def main():
             "tflops_kept_pairs": flop / (ms_step * 1e-3) / 1e12,
             "roofline": {"bound": "tensor", "kernel": "sparse_attn_fwd_kernel", "achieved": attn_tflops,
                          "peak": tc_peak, "unit": "TFLOP/s", "frac": attn_tflops / tc_peak,
-                         "peak_kind": f"{peak_kind} bf16 dense (burst)", "traffic": None,
-                         "flop_per_launch": flop},
+                         "peak_kind": f"{peak_kind} bf16 dense (burst)", "traffic": traffic,
+                         "traffic_source": traffic_src, "flop_per_launch": flop},
             "routing_roofline": {"bound": "hbm", "achieved": rbytes / (route_ms * 1e-3) / 1e9, "peak": hbm_peak,
                                  "unit": "GB/s", "frac": rbytes / (route_ms * 1e-3) / 1e9 / hbm_peak,
                                  "bytes_per_layer": rbytes},
