@@ -138,6 +138,23 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(self.samples), "source": "nvml, 20 ms"}
 
 
+# ----------------------------------------------------------------- ranks
+def max_over_ranks(value: float, device) -> float:
+    """Max of a per-rank timing over all ranks (identity when not distributed)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_ms_per_layer(max_total_ms: float, steps: int, world: int) -> float:
+    """Whole-job amortised ms per layer: each of `world` ranks runs one layer per step."""
+    return max_total_ms / steps / world
+
+
 # ----------------------------------------------------------------- helpers
 def kept_pair_count(off, n_chunks, sel, n_sel):
     """Kept token pairs of the layer from the GPU selection (host arithmetic)."""
@@ -302,11 +319,7 @@ def main():
         torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    total_ms = t0.elapsed_time(t1)
-    if world > 1:
-        tt = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        total_ms = float(tt.item())
+    total_ms = max_over_ranks(t0.elapsed_time(t1), dev)
     flags = binding.check_device_status()
     route_ms = statistics.median(a.elapsed_time(b) for a, b, _ in stages)
     attn_ms = statistics.median(b.elapsed_time(c) for _, b, c in stages)
@@ -344,12 +357,9 @@ def main():
             e2e_step()
         b.record(stream)
         torch.cuda.synchronize()
-        e2e_ms = a.elapsed_time(b) / args.steps
-        if world > 1:
-            tt = torch.tensor([e2e_ms], device=dev)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            e2e_ms = float(tt.item())
-        e2e = {"value": e2e_ms / world, "unit": "ms", "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+        e2e_ms = max_over_ranks(a.elapsed_time(b), dev)
+        e2e = {"value": job_ms_per_layer(e2e_ms, args.steps, world), "unit": "ms",
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
 
     # dense comparisons (not part of the timed value): the same kernels with
     # k = all causal chunks, and torch SDPA dense causal attention
@@ -388,7 +398,8 @@ def main():
 
     if rank == 0:
         line = {
-            "metric": METRIC, "value": ms_step / world, "unit": "ms", "n_gpus": world, "steps": args.steps,
+            "metric": METRIC, "value": job_ms_per_layer(total_ms, args.steps, world), "unit": "ms",
+            "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": False, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "L": w.L, "head_dim": 128,
