@@ -24,10 +24,11 @@
 //   key, -inf for a padding slot), so S already holds -inf there. Only tiles
 //   that hold keys of the diagonal chunk past the tile's first query row run
 //   a per-element causal compare (slot token <= query token).
-// * Warp roles (256 threads): warp 0 = TMA producer, warp 1 = tcgen05 MMA
-//   issuer (one thread), warp 2 = scheduler (resolves each work item's chunk
-//   list into a shared-memory ring up to 4 items ahead), warp 3 idle,
-//   warps 4-7 = softmax + epilogue (thread = query row = TMEM lane).
+// * Warp roles (256 threads): warp 0 = TMA producer of Q and K, warp 3 = TMA
+//   producer of V, warp 1 = tcgen05 MMA issuer (one thread), warp 2 =
+//   scheduler (resolves each work item's chunk list into a shared-memory ring
+//   up to 4 items ahead), warps 4-7 = softmax + epilogue (thread = query row
+//   = TMEM lane).
 // * Pipelines: Q double-buffered; separate K and V rings of 2 stages; a K
 //   stage is released as soon as its QK^T completes, a V stage after its PV.
 // * TMEM (512 columns): S double buffer (2 x 128 fp32 columns) and the O
@@ -140,8 +141,8 @@ static_assert(kSmemAlloc <= 227 * 1024, "shared memory budget");
 static_assert(OFF_BAR % 8 == 0 && OFF_SLOT % 16 == 0, "alignment");
 
 // role warps
-constexpr int W_PRODUCER = 0, W_MMA = 1, W_SCHED = 2, W_SOFTMAX0 = 4;
-constexpr int kSlotConsumers = 1 + 1 + 4;  // producer, MMA thread, 4 softmax warps
+constexpr int W_PRODUCER = 0, W_MMA = 1, W_SCHED = 2, W_VPRODUCER = 3, W_SOFTMAX0 = 4;
+constexpr int kSlotConsumers = 2 + 1 + 4;  // K and V producers, MMA thread, 4 softmax warps
 
 __device__ __forceinline__ int round8(int x) { return (x + 7) & ~7; }
 
@@ -283,8 +284,13 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_fwd_kernel(const __gr
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(B_SLFULL + sl));
     }
-  } else if (warp == W_PRODUCER) {
-    // ============================================================ producer
+  } else if (warp == W_PRODUCER || warp == W_VPRODUCER) {
+    // ============================================================ producers
+    // Two warps walk the same key stream: warp 0 loads Q and K (and writes
+    // each K stage's bias block and slot-token table), warp 3 loads V. A K
+    // stage frees when its QK^T completes and a V stage when its PV does;
+    // with separate warps the K loads never wait behind a V stage.
+    const bool kprod = warp == W_PRODUCER;
     uint32_t g = 0;  // global key-tile counter of this CTA
     int n_local = 0;
     for (int it = blockIdx.x; it < n_items; it += gridDim.x, ++n_local) {
@@ -293,12 +299,14 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_fwd_kernel(const __gr
       const ItemMeta M = slots[sl].m;
       const int2* seg_s = slots[sl].seg;
       const int ms = n_local & 1;
-      if (n_local >= 2 && !fl.wait(bar(B_QEMPTY + ms), ((n_local >> 1) - 1) & 1)) break;
-      if (lane == 0) {
-        mbar_arrive_expect_tx(bar(B_QFULL + ms), kTileBytes);
-        const uint32_t dq = sbase + OFF_Q + ms * kTileBytes;
-        tma_load_2d(dq, &maps.q, bar(B_QFULL + ms), 0, M.q_row0 + M.q0);
-        tma_load_2d(dq + kHalfBytes, &maps.q, bar(B_QFULL + ms), 64, M.q_row0 + M.q0);
+      if (kprod) {
+        if (n_local >= 2 && !fl.wait(bar(B_QEMPTY + ms), ((n_local >> 1) - 1) & 1)) break;
+        if (lane == 0) {
+          mbar_arrive_expect_tx(bar(B_QFULL + ms), kTileBytes);
+          const uint32_t dq = sbase + OFF_Q + ms * kTileBytes;
+          tma_load_2d(dq, &maps.q, bar(B_QFULL + ms), 0, M.q_row0 + M.q0);
+          tma_load_2d(dq + kHalfBytes, &maps.q, bar(B_QFULL + ms), 64, M.q_row0 + M.q0);
+        }
       }
       const int32_t* ob = p.off + (long long)M.b * (p.Nmax + 1);
       // chunk descriptors beyond SEG_CAP are read from global memory, 32 at a time
@@ -321,8 +329,12 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_fwd_kernel(const __gr
       bool ok = true;
       for (int kt = 0; kt < M.T; ++kt, ++g) {
         const int stk = g % NSK, stv = g % NSV, tk = g % NTOK;
-        if (g >= NSK && !fl.wait(bar(B_KEMPTY + stk), ((g / NSK) - 1) & 1)) { ok = false; break; }
-        if (g >= NTOK && !fl.wait(bar(B_TOKEMPTY + tk), ((g / NTOK) - 1) & 1)) { ok = false; break; }
+        if (kprod) {
+          if (g >= NSK && !fl.wait(bar(B_KEMPTY + stk), ((g / NSK) - 1) & 1)) { ok = false; break; }
+          if (g >= NTOK && !fl.wait(bar(B_TOKEMPTY + tk), ((g / NTOK) - 1) & 1)) { ok = false; break; }
+        } else {
+          if (g >= NSV && !fl.wait(bar(B_VEMPTY + stv), ((g / NSV) - 1) & 1)) { ok = false; break; }
+        }
         int* tok = slot_tok + tk * BN;
         unsigned char* bias = smem + OFF_BIAS + stk * kBiasBytes;
         // walk the key stream: lane b holds the b-th TMA box of this tile
@@ -333,12 +345,14 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_fwd_kernel(const __gr
           const int rows = min(dsc.y - seg_pos, BN - slot);
           const int groups = (rows + 7) >> 3;
           const int tok0 = dsc.x + seg_pos;
-          for (int s = lane; s < groups * 8; s += 32) {
-            const bool valid = s < rows;
-            tok[slot + s] = valid ? tok0 + s : kNoToken;
-            *reinterpret_cast<uint16_t*>(bias + noswz_off(slot + s, 0)) = valid ? 0 : kBf16NegInf;
+          if (kprod) {
+            for (int s = lane; s < groups * 8; s += 32) {
+              const bool valid = s < rows;
+              tok[slot + s] = valid ? tok0 + s : kNoToken;
+              *reinterpret_cast<uint16_t*>(bias + noswz_off(slot + s, 0)) = valid ? 0 : kBf16NegInf;
+            }
+            if (sq == M.nseg - 1 && tok0 + rows - 1 > M.q0) causal = 1;  // diagonal keys past the first query
           }
-          if (sq == M.nseg - 1 && tok0 + rows - 1 > M.q0) causal = 1;  // diagonal keys past the first query
           // the whole piece in one box per head-dim half (per-op TMA cost
           // dominates for small boxes, so never split a piece)
           if (lane == nbox) {
@@ -355,30 +369,32 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_fwd_kernel(const __gr
             ++sq;
           }
         }
-        for (int s = slot + lane; s < BN; s += 32) {
-          tok[s] = kNoToken;
-          *reinterpret_cast<uint16_t*>(bias + noswz_off(s, 0)) = kBf16NegInf;
-        }
-        if (lane == 0) tile_flag[tk] = causal;
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(bar(B_TOKFULL + tk));
-          mbar_arrive_expect_tx(bar(B_KFULL + stk), bytes);
-        }
-        __syncwarp();
-        const uint32_t dk = sbase + OFF_K + stk * kTileBytes;
-        if (lane < nbox) {
-          tma_load_2d(dk + my_so, &maps.k[my_bx], bar(B_KFULL + stk), 0, my_y);
-          tma_load_2d(dk + kHalfBytes + my_so, &maps.k[my_bx], bar(B_KFULL + stk), 64, my_y);
-        }
-        if (g >= NSV && !fl.wait(bar(B_VEMPTY + stv), ((g / NSV) - 1) & 1)) { ok = false; ++g; break; }
-        if (lane == 0) mbar_arrive_expect_tx(bar(B_VFULL + stv), bytes);
-        __syncwarp();
-        const uint32_t dv = sbase + OFF_V + stv * kTileBytes;
-        if (lane < nbox) {
-          tma_load_2d(dv + my_so, &maps.v[my_bx], bar(B_VFULL + stv), 0, my_y);
-          tma_load_2d(dv + kHalfBytes + my_so, &maps.v[my_bx], bar(B_VFULL + stv), 64, my_y);
+        if (kprod) {
+          for (int s = slot + lane; s < BN; s += 32) {
+            tok[s] = kNoToken;
+            *reinterpret_cast<uint16_t*>(bias + noswz_off(s, 0)) = kBf16NegInf;
+          }
+          if (lane == 0) tile_flag[tk] = causal;
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive(bar(B_TOKFULL + tk));
+            mbar_arrive_expect_tx(bar(B_KFULL + stk), bytes);
+          }
+          __syncwarp();
+          const uint32_t dk = sbase + OFF_K + stk * kTileBytes;
+          if (lane < nbox) {
+            tma_load_2d(dk + my_so, &maps.k[my_bx], bar(B_KFULL + stk), 0, my_y);
+            tma_load_2d(dk + kHalfBytes + my_so, &maps.k[my_bx], bar(B_KFULL + stk), 64, my_y);
+          }
+        } else {
+          if (lane == 0) mbar_arrive_expect_tx(bar(B_VFULL + stv), bytes);
+          __syncwarp();
+          const uint32_t dv = sbase + OFF_V + stv * kTileBytes;
+          if (lane < nbox) {
+            tma_load_2d(dv + my_so, &maps.v[my_bx], bar(B_VFULL + stv), 0, my_y);
+            tma_load_2d(dv + kHalfBytes + my_so, &maps.v[my_bx], bar(B_VFULL + stv), 64, my_y);
+          }
         }
       }
       __syncwarp();
@@ -387,12 +403,15 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_fwd_kernel(const __gr
     }
     // drain: every copy this warp issued must have landed before teardown
     if (lane == 0) {
-      for (uint32_t gg = (g > NSK ? g - NSK : 0); gg < g; ++gg)
-        mbar_wait(bar(B_KFULL + gg % NSK), (gg / NSK) & 1, kWaitLimitNs);
-      for (uint32_t gg = (g > NSV ? g - NSV : 0); gg < g; ++gg)
-        mbar_wait(bar(B_VFULL + gg % NSV), (gg / NSV) & 1, kWaitLimitNs);
-      for (int n = (n_local > 2 ? n_local - 2 : 0); n < n_local; ++n)
-        mbar_wait(bar(B_QFULL + (n & 1)), (n >> 1) & 1, kWaitLimitNs);
+      if (kprod) {
+        for (uint32_t gg = (g > NSK ? g - NSK : 0); gg < g; ++gg)
+          mbar_wait(bar(B_KFULL + gg % NSK), (gg / NSK) & 1, kWaitLimitNs);
+        for (int n = (n_local > 2 ? n_local - 2 : 0); n < n_local; ++n)
+          mbar_wait(bar(B_QFULL + (n & 1)), (n >> 1) & 1, kWaitLimitNs);
+      } else {
+        for (uint32_t gg = (g > NSV ? g - NSV : 0); gg < g; ++gg)
+          mbar_wait(bar(B_VFULL + gg % NSV), (gg / NSV) & 1, kWaitLimitNs);
+      }
     }
   } else if (warp == W_MMA) {
     // ============================================================ MMA issuer
