@@ -22,23 +22,36 @@
 // * Masking: padding slots are removed inside the tensor core. Every QK^T
 //   gets one extra K=16 MMA step, ones-column x per-slot bias (0 for a kept
 //   key, -inf for a padding slot), so S already holds -inf there. Only tiles
-//   that hold keys of the diagonal chunk past the tile's first query row run
-//   a per-element causal compare (slot token <= query token).
-// * Warp roles (256 threads): warp 0 = TMA producer of Q and K, warp 3 = TMA
-//   producer of V, warp 1 = tcgen05 MMA issuer (one thread), warp 2 =
-//   scheduler (resolves each work item's chunk list into a shared-memory ring
-//   up to 4 items ahead), warps 4-7 = softmax + epilogue (thread = query row
-//   = TMEM lane).
+//   that hold keys of the diagonal chunk past the tile's first query row
+//   mask causally: that piece is the tile's last and its slots hold
+//   consecutive tokens, so a row masks the slots from one threshold on.
+// * Warp roles (512 threads, four warpgroups): warp 0 = TMA producer of Q
+//   and K (and of the bias blocks), warp 3 = TMA producer of V, warp 1 =
+//   QK^T issuer, warp 14 = PV issuer (one thread each), warp 2 = scheduler
+//   (resolves each work item's chunk list into a shared-memory ring up to 4
+//   items ahead), warps 4-11 = softmax + epilogue: warpgroup 1 takes key
+//   slots 0..63 of every tile and warpgroup 2 slots 64..127, two warps per
+//   TMEM lane quarter (thread = query row = TMEM lane). Warpgroups 0 and 3
+//   hand their registers to the softmax warpgroups (setmaxnreg). The two
+//   issuers sit on sub-partitions apart from the K producer: an issuer that
+//   shares one with the K producer measurably slows that sub-partition's
+//   softmax warps.
 // * Pipelines: Q double-buffered; separate K and V rings of 2 stages; a K
 //   stage is released as soon as its QK^T completes, a V stage after its PV.
-// * TMEM (512 columns): S double buffer (2 x 128 fp32 columns) and the O
+//   With two issuing threads the tensor pipe keeps work queued while either
+//   one waits on a barrier.
+// * TMEM (512 columns): three S buffers (3 x 128 fp32 columns) and the O
 //   accumulator (128 columns). P (bf16) is written back into the S buffer it
-//   came from and consumed from TMEM by the PV MMA (A in TMEM, V as an
-//   N-major shared-memory operand).
-// * Online softmax in the log2 domain; the running max is only raised (and O
-//   rescaled in TMEM) when it grows by more than 8 (a factor 256), which keeps
-//   O / l exact while skipping nearly all rescales; only then does the softmax
-//   wait for the previous PV.
+//   came from, each warp into its own half, and consumed from TMEM by the PV
+//   MMA (A in TMEM, V as an N-major shared-memory operand). The QK^T issuer
+//   runs up to three tiles ahead of the PV.
+// * Online softmax in the log2 domain. The two warps of a lane quarter trade
+//   their half-row maxima through shared memory once per tile, then each
+//   exponentiates its 64 columns and keeps its own partial row sum (the two
+//   are added in the epilogue). The running max is only raised (and O
+//   rescaled in TMEM, each warp its half of the columns) when it grows by
+//   more than 8 (a factor 256), which keeps O / l exact while skipping nearly
+//   all rescales; only then does the softmax wait for the previous PV.
 // * Every mbarrier wait is bounded; a timeout sets DHSA_DEVFLAG_WAIT_TIMEOUT,
 //   the CTA drains its own in-flight copies and MMAs (again bounded), frees
 //   its TMEM and exits.
@@ -56,16 +69,16 @@ constexpr int BM = 128;              // query rows per tile
 constexpr int BN = 128;              // key slots per tile
 constexpr int NSK = 2;               // K pipeline stages
 constexpr int NSV = 2;               // V pipeline stages
+constexpr int NSB = 3;               // S/P buffers in TMEM
 constexpr int NTOK = 4;              // slot-token table ring (causal tiles)
 constexpr int NSLOT = 4;             // scheduled work items in flight
 constexpr int SEG_CAP = 64;          // chunk descriptors kept in shared memory per item
-constexpr int kThreads = 256;
+constexpr int kThreads = 512;
 constexpr uint32_t kHalfBytes = 128 * 128;   // 128 rows x 64 bf16 (one 128B-swizzled half tile)
 constexpr uint32_t kTileBytes = 2 * kHalfBytes;
 constexpr uint32_t kBiasBytes = 128 * 16 * 2;  // 128 rows x 16 bf16, no swizzle
 constexpr uint32_t kTmemCols = 512;
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s per wait
-constexpr int kNoToken = 0x7fffffff;
 constexpr uint16_t kBf16One = 0x3F80, kBf16NegInf = 0xFF80;
 
 struct AttnMaps {
@@ -111,27 +124,29 @@ constexpr uint32_t OFF_K = OFF_Q + 2 * kTileBytes;              // NSK x 32 KB
 constexpr uint32_t OFF_V = OFF_K + NSK * kTileBytes;            // NSV x 32 KB
 constexpr uint32_t OFF_ONES = OFF_V + NSV * kTileBytes;         // 4 KB
 constexpr uint32_t OFF_BIAS = OFF_ONES + kBiasBytes;            // NSK x 4 KB
-constexpr uint32_t OFF_TOK = OFF_BIAS + NSK * kBiasBytes;       // NTOK x 128 int
-constexpr uint32_t OFF_FLAG = OFF_TOK + NTOK * BN * 4;          // NTOK int
-constexpr uint32_t OFF_SLOT = OFF_FLAG + 16 * ((NTOK * 4 + 15) / 16);
-constexpr uint32_t OFF_BAR = OFF_SLOT + NSLOT * sizeof(ItemSlot);
+constexpr uint32_t OFF_TINFO = OFF_BIAS + NSK * kBiasBytes;    // NTOK int4 tile descriptors
+constexpr uint32_t OFF_SLOT = OFF_TINFO + NTOK * 16;
+constexpr uint32_t OFF_XCHG = OFF_SLOT + NSLOT * sizeof(ItemSlot);   // 2 x 2 x 128 floats, twice
+constexpr uint32_t OFF_BAR = OFF_XCHG + 2 * 2 * 2 * BM * 4;
 enum {
   B_QFULL = 0,
   B_QEMPTY = B_QFULL + 2,
   B_SLFULL = B_QEMPTY + 2,
   B_SLEMPTY = B_SLFULL + NSLOT,
   B_KFULL = B_SLEMPTY + NSLOT,
-  B_KEMPTY = B_KFULL + NSK,
-  B_VFULL = B_KEMPTY + NSK,
-  B_VEMPTY = B_VFULL + NSV,
-  B_TOKFULL = B_VEMPTY + NSV,
+  B_VFULL = B_KFULL + NSK,
+  B_TOKFULL = B_VFULL + NSV,
   B_TOKEMPTY = B_TOKFULL + NTOK,
-  B_SFULL = B_TOKEMPTY + NTOK,
-  B_PREADY = B_SFULL + 2,
-  B_ODONE = B_PREADY + 2,
-  B_OFINAL = B_ODONE + 1,
+  B_SFULL = B_TOKEMPTY + NTOK,   // QK^T(g) complete: S ready, K stage and bias block free
+  B_PREADY = B_SFULL + NSB,
+  B_PVDONE = B_PREADY + NSB,     // PV(g) complete: P buffer and V stage free, O current
+  B_OFINAL = B_PVDONE + NSB,
   B_FINAL = B_OFINAL + 1,
-  B_COUNT = B_FINAL + 1
+  B_FINALPV = B_FINAL + 1,
+  B_XMAX = B_FINALPV + 1,        // [quarter][tile parity]: the softmax pair's row-max exchange
+  B_XSUM = B_XMAX + 8,           // [quarter][item parity]: the pair's row-sum exchange
+  B_TEARDOWN = B_XSUM + 8,
+  B_COUNT = B_TEARDOWN + 1
 };
 constexpr uint32_t OFF_TMEMPTR = OFF_BAR + 8 * B_COUNT;
 constexpr uint32_t OFF_ABORT = OFF_TMEMPTR + 4;
@@ -141,8 +156,15 @@ static_assert(kSmemAlloc <= 227 * 1024, "shared memory budget");
 static_assert(OFF_BAR % 8 == 0 && OFF_SLOT % 16 == 0, "alignment");
 
 // role warps
-constexpr int W_PRODUCER = 0, W_MMA = 1, W_SCHED = 2, W_VPRODUCER = 3, W_SOFTMAX0 = 4;
-constexpr int kSlotConsumers = 2 + 1 + 4;  // K and V producers, MMA thread, 4 softmax warps
+constexpr int W_PRODUCER = 0, W_MMA = 1, W_SCHED = 2, W_VPRODUCER = 3, W_SOFTMAX0 = 4, W_PV = 14;
+constexpr int kSoftmaxWarps = 8;
+constexpr int kSlotConsumers = 2 + 2 + kSoftmaxWarps;  // K and V producers, QK and PV issuers, softmax warps
+// registers per thread after reallocation: warpgroup 0 (producers, scheduler,
+// QK issuer) and warpgroup 3 (PV issuer) give theirs to the two softmax
+// warpgroups
+constexpr uint32_t kRegsLaunch = 65536 / kThreads / 8 * 8;   // 128 at 512 threads
+constexpr uint32_t kRegsWg0 = 96, kRegsWg3 = 64, kRegsSoftmax = 176;
+static_assert(128 * (kRegsWg0 + kRegsWg3 + 2 * kRegsSoftmax) <= kRegsLaunch * kThreads, "register split");
 
 __device__ __forceinline__ int round8(int x) { return (x + 7) & ~7; }
 
@@ -180,8 +202,8 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_fwd_kernel(const __gr
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
-  int* slot_tok = reinterpret_cast<int*>(smem + OFF_TOK);
-  int* tile_flag = reinterpret_cast<int*>(smem + OFF_FLAG);
+  // per key tile: (causal, first slot of the diagonal piece, that slot minus its token)
+  int4* tile_info = reinterpret_cast<int4*>(smem + OFF_TINFO);
   ItemSlot* slots = reinterpret_cast<ItemSlot*>(smem + OFF_SLOT);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_ABORT);
   auto bar = [&](int idx) { return sbase + OFF_BAR + 8u * idx; };
@@ -196,28 +218,30 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_fwd_kernel(const __gr
       for (int s = 0; s < 2; ++s) {
         mbar_init(bar(B_QFULL + s), 1);
         mbar_init(bar(B_QEMPTY + s), 1);
+      }
+      for (int s = 0; s < NSB; ++s) {
         mbar_init(bar(B_SFULL + s), 1);
-        mbar_init(bar(B_PREADY + s), 4);
+        mbar_init(bar(B_PREADY + s), kSoftmaxWarps);
+        mbar_init(bar(B_PVDONE + s), 1);
       }
       for (int s = 0; s < NSLOT; ++s) {
         mbar_init(bar(B_SLFULL + s), 1);
         mbar_init(bar(B_SLEMPTY + s), kSlotConsumers);
       }
-      for (int s = 0; s < NSK; ++s) {
-        mbar_init(bar(B_KFULL + s), 1);
-        mbar_init(bar(B_KEMPTY + s), 1);
-      }
-      for (int s = 0; s < NSV; ++s) {
-        mbar_init(bar(B_VFULL + s), 1);
-        mbar_init(bar(B_VEMPTY + s), 1);
-      }
+      for (int s = 0; s < NSK; ++s) mbar_init(bar(B_KFULL + s), 1);
+      for (int s = 0; s < NSV; ++s) mbar_init(bar(B_VFULL + s), 1);
       for (int s = 0; s < NTOK; ++s) {
         mbar_init(bar(B_TOKFULL + s), 1);
-        mbar_init(bar(B_TOKEMPTY + s), 4);
+        mbar_init(bar(B_TOKEMPTY + s), kSoftmaxWarps);
       }
-      mbar_init(bar(B_ODONE), 1);
       mbar_init(bar(B_OFINAL), 1);
       mbar_init(bar(B_FINAL), 1);
+      mbar_init(bar(B_FINALPV), 1);
+      for (int s = 0; s < 8; ++s) {
+        mbar_init(bar(B_XMAX + s), 2);
+        mbar_init(bar(B_XSUM + s), 2);
+      }
+      mbar_init(bar(B_TEARDOWN), kThreads / 32 - 1);
       fence_mbar_init();
       prefetch_tmap(&maps.q);
       for (int s = 0; s < 16; ++s) {
@@ -233,7 +257,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_fwd_kernel(const __gr
   // get -inf added; a masked V row is multiplied by P = 0): zero every K and
   // V stage and the bias blocks once; then write the ones column of the bias
   // step's A operand.
-  for (uint32_t o = threadIdx.x * 16; o < OFF_TOK - OFF_K; o += kThreads * 16)
+  for (uint32_t o = threadIdx.x * 16; o < OFF_TINFO - OFF_K; o += kThreads * 16)
     *reinterpret_cast<uint4*>(smem + OFF_K + o) = make_uint4(0, 0, 0, 0);
   __syncthreads();
   if (threadIdx.x < BM) *reinterpret_cast<uint16_t*>(smem + OFF_ONES + noswz_off(threadIdx.x, 0)) = kBf16One;
@@ -243,6 +267,8 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_fwd_kernel(const __gr
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + OFF_TMEMPTR);
   Flags fl{abort_flag, p.status};
+  if (warp < W_SOFTMAX0) regs_dec<kRegsWg0>();
+  else if (warp >= W_SOFTMAX0 + kSoftmaxWarps) regs_dec<kRegsWg3>();
 
   if (warp == W_SCHED) {
     // ============================================================ scheduler
@@ -330,15 +356,16 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_fwd_kernel(const __gr
       for (int kt = 0; kt < M.T; ++kt, ++g) {
         const int stk = g % NSK, stv = g % NSV, tk = g % NTOK;
         if (kprod) {
-          if (g >= NSK && !fl.wait(bar(B_KEMPTY + stk), ((g / NSK) - 1) & 1)) { ok = false; break; }
+          // the K stage (and its bias block) of tile g - NSK is free once that QK^T is done
+          if (g >= NSK && !fl.wait(bar(B_SFULL + (g - NSK) % NSB), ((g - NSK) / NSB) & 1)) { ok = false; break; }
           if (g >= NTOK && !fl.wait(bar(B_TOKEMPTY + tk), ((g / NTOK) - 1) & 1)) { ok = false; break; }
         } else {
-          if (g >= NSV && !fl.wait(bar(B_VEMPTY + stv), ((g / NSV) - 1) & 1)) { ok = false; break; }
+          // the V stage of tile g - NSV is free once that PV is done
+          if (g >= NSV && !fl.wait(bar(B_PVDONE + (g - NSV) % NSB), ((g - NSV) / NSB) & 1)) { ok = false; break; }
         }
-        int* tok = slot_tok + tk * BN;
         unsigned char* bias = smem + OFF_BIAS + stk * kBiasBytes;
         // walk the key stream: lane b holds the b-th TMA box of this tile
-        int slot = 0, causal = 0, nbox = 0, my_y = 0, my_so = 0, my_bx = 0;
+        int slot = 0, causal = 0, d_slot = 0, d_off = 0, nbox = 0, my_y = 0, my_so = 0, my_bx = 0;
         uint32_t bytes = 0;
         while (slot < BN && sq < M.nseg) {
           const int2 dsc = desc(sq);
@@ -346,12 +373,15 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_fwd_kernel(const __gr
           const int groups = (rows + 7) >> 3;
           const int tok0 = dsc.x + seg_pos;
           if (kprod) {
-            for (int s = lane; s < groups * 8; s += 32) {
-              const bool valid = s < rows;
-              tok[slot + s] = valid ? tok0 + s : kNoToken;
-              *reinterpret_cast<uint16_t*>(bias + noswz_off(slot + s, 0)) = valid ? 0 : kBf16NegInf;
+            for (int s = lane; s < groups * 8; s += 32)
+              *reinterpret_cast<uint16_t*>(bias + noswz_off(slot + s, 0)) = s < rows ? 0 : kBf16NegInf;
+            if (sq == M.nseg - 1 && tok0 + rows - 1 > M.q0) {
+              // diagonal keys past the first query: the piece is the tile's
+              // last, slot s >= d_slot holds token s - d_off
+              causal = 1;
+              d_slot = slot;
+              d_off = slot - tok0;
             }
-            if (sq == M.nseg - 1 && tok0 + rows - 1 > M.q0) causal = 1;  // diagonal keys past the first query
           }
           // the whole piece in one box per head-dim half (per-op TMA cost
           // dominates for small boxes, so never split a piece)
@@ -370,11 +400,9 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_fwd_kernel(const __gr
           }
         }
         if (kprod) {
-          for (int s = slot + lane; s < BN; s += 32) {
-            tok[s] = kNoToken;
+          for (int s = slot + lane; s < BN; s += 32)
             *reinterpret_cast<uint16_t*>(bias + noswz_off(s, 0)) = kBf16NegInf;
-          }
-          if (lane == 0) tile_flag[tk] = causal;
+          if (lane == 0) tile_info[tk] = make_int4(causal, d_slot, d_off, 0);
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
@@ -414,30 +442,15 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_fwd_kernel(const __gr
       }
     }
   } else if (warp == W_MMA) {
-    // ============================================================ MMA issuer
+    // ============================================================ QK^T issuer
+    // S[g % NSB] = Q K(g)^T (+ ones x bias). The buffer last held P(g - NSB),
+    // so it is reused once PV(g - NSB) has completed.
     if (lane == 0) {
       const uint32_t idesc_qk = idesc_bf16_f32(BM, BN, false);
-      const uint32_t idesc_pv = idesc_bf16_f32(BM, 128, true);
-      const uint32_t tS0 = tmem, tO = tmem + 256;
+      const uint32_t tS0 = tmem;
       const uint64_t ones_desc = smem_desc_noswz(sbase + OFF_ONES, 128, 256);
       uint32_t g = 0;
       int n_local = 0;
-      auto issue_pv = [&](uint32_t u, bool first, bool last) -> bool {
-        const int stv = u % NSV, sb = u & 1;
-        if (!fl.wait(bar(B_PREADY + sb), (u >> 1) & 1)) return false;
-        if (!fl.wait(bar(B_VFULL + stv), (u / NSV) & 1)) return false;
-        tc_fence_after();
-        const uint32_t v0 = sbase + OFF_V + stv * kTileBytes;
-#pragma unroll
-        for (int ks = 0; ks < BN / 16; ++ks) {
-          const uint64_t bdesc = smem_desc_sw128(v0 + ks * 2048, kHalfBytes, 1024);
-          mma_ts(tO, tS0 + sb * 128 + ks * 8, bdesc, idesc_pv, (!first || ks > 0) ? 1u : 0u);
-        }
-        mma_commit(bar(B_VEMPTY + stv));
-        mma_commit(bar(B_ODONE));
-        if (last) mma_commit(bar(B_OFINAL));
-        return true;
-      };
       for (int it = blockIdx.x; it < n_items; it += gridDim.x, ++n_local) {
         const int sl = n_local % NSLOT;
         if (!fl.wait(bar(B_SLFULL + sl), (n_local / NSLOT) & 1)) break;
@@ -448,8 +461,9 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_fwd_kernel(const __gr
         const uint32_t qa = sbase + OFF_Q + ms * kTileBytes;
         bool ok = true;
         for (int kt = 0; kt < T; ++kt, ++g) {
-          const int stk = g % NSK, sb = g & 1;
+          const int stk = g % NSK, sb = g % NSB;
           if (!fl.wait(bar(B_KFULL + stk), (g / NSK) & 1)) { ok = false; break; }
+          if (g >= NSB && !fl.wait(bar(B_PVDONE + sb), ((g / NSB) - 1) & 1)) { ok = false; break; }
           tc_fence_after();
           const uint32_t k0 = sbase + OFF_K + stk * kTileBytes;
 #pragma unroll
@@ -461,29 +475,68 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_fwd_kernel(const __gr
           // S += ones x bias: -inf on padding slots
           mma_ss(tS0 + sb * 128, ones_desc, smem_desc_noswz(sbase + OFF_BIAS + stk * kBiasBytes, 128, 256),
                  idesc_qk, 1u);
-          mma_commit(bar(B_KEMPTY + stk));
           mma_commit(bar(B_SFULL + sb));
           if (kt == T - 1) mma_commit(bar(B_QEMPTY + ms));
-          if (kt >= 1 && !issue_pv(g - 1, kt == 1, false)) { ok = false; break; }
         }
         if (!ok) break;
-        if (T == 0) {
-          mma_commit(bar(B_QEMPTY + ms));   // an empty key set: nothing to multiply
-          mma_commit(bar(B_OFINAL));
-        } else if (!issue_pv(g - 1, T == 1, true)) {
-          break;
-        }
+        if (T == 0) mma_commit(bar(B_QEMPTY + ms));   // an empty key set: nothing to multiply
       }
-      // drain the tensor pipe before TMEM is released
+      // drain this thread's tensor work before TMEM is released
       mma_commit(bar(B_FINAL));
       mbar_wait(bar(B_FINAL), 0, kWaitLimitNs);
     }
-  } else if (warp >= W_SOFTMAX0) {
+  } else if (warp == W_PV) {
+    // ============================================================ PV issuer
+    // O += P(g) V(g), P read from TMEM where the softmax left it. A second
+    // issuing thread keeps the tensor pipe fed while the QK^T issuer waits.
+    if (lane == 0) {
+      const uint32_t idesc_pv = idesc_bf16_f32(BM, 128, true);
+      const uint32_t tS0 = tmem, tO = tmem + 384;
+      uint32_t g = 0;
+      int n_local = 0;
+      for (int it = blockIdx.x; it < n_items; it += gridDim.x, ++n_local) {
+        const int sl = n_local % NSLOT;
+        if (!fl.wait(bar(B_SLFULL + sl), (n_local / NSLOT) & 1)) break;
+        const int T = slots[sl].m.T;
+        mbar_arrive(bar(B_SLEMPTY + sl));
+        bool ok = true;
+        for (int kt = 0; kt < T; ++kt, ++g) {
+          const int stv = g % NSV, sb = g % NSB;
+          if (!fl.wait(bar(B_PREADY + sb), (g / NSB) & 1)) { ok = false; break; }
+          if (!fl.wait(bar(B_VFULL + stv), (g / NSV) & 1)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t v0 = sbase + OFF_V + stv * kTileBytes;
+#pragma unroll
+          for (int ks = 0; ks < BN / 16; ++ks) {
+            const uint64_t bdesc = smem_desc_sw128(v0 + ks * 2048, kHalfBytes, 1024);
+            // P of key slots 0..63 sits in S columns 0..31, of slots 64..127 in 64..95
+            mma_ts(tO, tS0 + sb * 128 + (ks >> 2) * 64 + (ks & 3) * 8, bdesc, idesc_pv,
+                   (kt > 0 || ks > 0) ? 1u : 0u);
+          }
+          mma_commit(bar(B_PVDONE + sb));
+          if (kt == T - 1) mma_commit(bar(B_OFINAL));
+        }
+        if (!ok) break;
+        if (T == 0) mma_commit(bar(B_OFINAL));
+      }
+      mma_commit(bar(B_FINALPV));
+      mbar_wait(bar(B_FINALPV), 0, kWaitLimitNs);
+    }
+  } else if (warp >= W_SOFTMAX0 && warp < W_SOFTMAX0 + 8) {
     // ============================================================ softmax + epilogue
+    // Two warps per TMEM lane quarter: warpgroup 1 takes key slots 0..63 of
+    // every tile, warpgroup 2 slots 64..127 (so each SM sub-partition runs two
+    // softmax warps). The pair agrees on the row max through shared memory
+    // once per tile; each keeps its own partial row sum and rescales and
+    // writes its own half of the O columns.
     const int quarter = warp & 3;             // TMEM lanes 32*quarter .. +31
+    const int half = (warp - W_SOFTMAX0) >> 2;
+    regs_inc<kRegsSoftmax>();
     const int row = quarter * 32 + lane;      // query row within the tile
     const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
-    const uint32_t tS0 = tmem + lane_addr, tO = tmem + lane_addr + 256;
+    const uint32_t tS0 = tmem + lane_addr + half * 64, tO = tmem + lane_addr + 384 + half * 64;
+    float* xmax = reinterpret_cast<float*>(smem + OFF_XCHG);    // [buffer][half][row]
+    float* xsum = xmax + 2 * 2 * BM;                             // [buffer][half][row]
     const float c = p.scale_log2;
     uint32_t g = 0;
     int n_local = 0;
@@ -497,48 +550,53 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_fwd_kernel(const __gr
       float m_used = -INFINITY, l_sum = 0.f;
       bool ok = true;
       for (int kt = 0; kt < M.T; ++kt, ++g) {
-        const int sb = g & 1, tk = g % NTOK;
-        if (!fl.wait(bar(B_SFULL + sb), (g >> 1) & 1) || !fl.wait(bar(B_TOKFULL + tk), (g / NTOK) & 1)) {
+        const int sb = g % NSB, tk = g % NTOK, xb = g & 1;
+        if (!fl.wait(bar(B_SFULL + sb), (g / NSB) & 1) || !fl.wait(bar(B_TOKFULL + tk), (g / NTOK) & 1)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        uint32_t s[BN];
+        uint32_t s[64];
         tmem_ld32(tS0 + sb * 128 + 0, *reinterpret_cast<uint32_t(*)[32]>(s + 0));
         tmem_ld32(tS0 + sb * 128 + 32, *reinterpret_cast<uint32_t(*)[32]>(s + 32));
-        tmem_ld32(tS0 + sb * 128 + 64, *reinterpret_cast<uint32_t(*)[32]>(s + 64));
-        tmem_ld32(tS0 + sb * 128 + 96, *reinterpret_cast<uint32_t(*)[32]>(s + 96));
         tmem_wait_ld();
-        if (tile_flag[tk]) {
-          const int4* tok4 = reinterpret_cast<const int4*>(slot_tok + tk * BN);
+        const int4 ti = tile_info[tk];
+        if (ti.x) {
+          // keys after query token qt: the slots from thr on (slots past the
+          // diagonal piece are padding and already -inf)
+          const int thr = max(qt + ti.z + 1, ti.y) - half * 64;
 #pragma unroll
-          for (int c4 = 0; c4 < BN / 4; ++c4) {
-            const int4 tq = tok4[c4];
-            if (tq.x > qt) s[4 * c4 + 0] = __float_as_uint(-INFINITY);
-            if (tq.y > qt) s[4 * c4 + 1] = __float_as_uint(-INFINITY);
-            if (tq.z > qt) s[4 * c4 + 2] = __float_as_uint(-INFINITY);
-            if (tq.w > qt) s[4 * c4 + 3] = __float_as_uint(-INFINITY);
-          }
+          for (int e = 0; e < 64; ++e)
+            if (e >= thr) s[e] = __float_as_uint(-INFINITY);
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(B_TOKEMPTY + tk));
-        // row max over raw scores, 8 independent chains
+        // row max over this half, 8 independent chains
         float mx8[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) mx8[e] = __uint_as_float(s[e]);
 #pragma unroll
-        for (int cc = 8; cc < BN; ++cc) mx8[cc & 7] = fmaxf(mx8[cc & 7], __uint_as_float(s[cc]));
-        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+        for (int cc = 8; cc < 64; ++cc) mx8[cc & 7] = fmaxf(mx8[cc & 7], __uint_as_float(s[cc]));
+        float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                         fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+        // exchange the half-row maxima with the partner warp (same rows)
+        xmax[(xb * 2 + half) * BM + row] = mx;
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(bar(B_TOKEMPTY + tk));
+          mbar_arrive(bar(B_XMAX + quarter * 2 + xb));
+        }
+        if (!fl.wait(bar(B_XMAX + quarter * 2 + xb), (g >> 1) & 1)) { ok = false; break; }
+        tc_fence_after();
+        mx = fmaxf(mx, xmax[(xb * 2 + (half ^ 1)) * BM + row]);
         const float m_new = fmaxf(m_used, mx * c);
         const bool rescale = m_new > m_used + 8.0f;  // also true on the first tile
         if (kt > 0 && __any_sync(0xffffffffu, rescale)) {
           // O may only be touched once the previous tile's PV has finished
-          if (!fl.wait(bar(B_ODONE), (g - 1) & 1)) { ok = false; break; }
+          if (!fl.wait(bar(B_PVDONE + (g - 1) % NSB), ((g - 1) / NSB) & 1)) { ok = false; break; }
           tc_fence_after();
           const float f = rescale ? fast_exp2(m_used - m_new) : 1.f;
 #pragma unroll
-          for (int c4 = 0; c4 < 4; ++c4) {
+          for (int c4 = 0; c4 < 2; ++c4) {
             uint32_t o[32];
             tmem_ld32(tO + 32 * c4, o);
             tmem_wait_ld();
@@ -550,35 +608,42 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_fwd_kernel(const __gr
           if (rescale) l_sum *= f;
         }
         if (rescale) m_used = m_new;
-        const float neg_m = -m_used;
+        // a row whose keys so far are all masked keeps m = -inf: its p are 0
+        const float neg_m = m_used == -INFINITY ? 0.f : -m_used;
         float rs8[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) rs8[e] = 0.f;
-        uint32_t pk[BN / 2];
+        uint32_t pk[32];
 #pragma unroll
-        for (int cc = 0; cc < BN / 2; ++cc) {
+        for (int cc = 0; cc < 32; ++cc) {
           const float p0 = fast_exp2(fmaf(__uint_as_float(s[2 * cc]), c, neg_m));
           const float p1 = fast_exp2(fmaf(__uint_as_float(s[2 * cc + 1]), c, neg_m));
           rs8[cc & 7] += p0 + p1;
           pk[cc] = pack_bf16x2(p0, p1);
         }
         l_sum += ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
-        tmem_st32(tS0 + sb * 128 + 0, *reinterpret_cast<uint32_t(*)[32]>(pk + 0));
-        tmem_st32(tS0 + sb * 128 + 32, *reinterpret_cast<uint32_t(*)[32]>(pk + 32));
+        // P (bf16 pairs) over the first 32 of this half's 64 S columns
+        tmem_st32(tS0 + sb * 128, pk);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(B_PREADY + sb));
       }
       if (!ok) break;
-      // epilogue: O / l -> bf16 (an empty key set, which valid CSR input never
-      // has, writes zeros)
+      // epilogue: O / l -> bf16 over this warp's 64 columns (an empty key
+      // set, which valid CSR input never has, writes zeros)
+      const int lb = n_local & 1;
+      xsum[(lb * 2 + half) * BM + row] = l_sum;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(B_XSUM + quarter * 2 + lb));
+      if (!fl.wait(bar(B_XSUM + quarter * 2 + lb), (n_local >> 1) & 1)) break;
+      const float l_tot = l_sum + xsum[(lb * 2 + (half ^ 1)) * BM + row];
       if (!fl.wait(bar(B_OFINAL), n_local & 1)) break;
       tc_fence_after();
-      const float inv_l = M.T > 0 ? 1.f / l_sum : 0.f;
-      __nv_bfloat16* orow = p.O + ((long long)M.q_row0 + qt) * kHeadDim;
+      const float inv_l = M.T > 0 ? 1.f / l_tot : 0.f;
+      __nv_bfloat16* orow = p.O + ((long long)M.q_row0 + qt) * kHeadDim + half * 64;
 #pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4) {
+      for (int c4 = 0; c4 < 2; ++c4) {
         uint32_t o[32];
         tmem_ld32(tO + 32 * c4, o);
         tmem_wait_ld();
@@ -604,11 +669,18 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_fwd_kernel(const __gr
   }
 
   // ---------------------------------------------------------------- teardown
+  // Every warp reports to one mbarrier and exits; warp 1, which allocated
+  // TMEM, frees it once all the others (and its own MMAs) are done.
   __syncwarp();  // lanes that waited out their role's single-thread work reconverge here
   tc_fence_before();
-  __syncthreads();
+  if (warp != W_MMA) {
+    if (lane == 0) mbar_arrive(bar(B_TEARDOWN));
+    return;
+  }
+  mbar_wait(bar(B_TEARDOWN), 0, kWaitLimitNs);
+  __syncwarp();
   tc_fence_after();
-  if (warp == W_MMA) tmem_dealloc(tmem, kTmemCols);
+  tmem_dealloc(tmem, kTmemCols);
 }
 
 // Work list: one item per (b, hq, chunk i, 128-row tile of i), ordered
