@@ -31,8 +31,10 @@ Parity pins: every function here is pinned by tests under tests/ to values
 fixed independently of this file (hand-computed pooling cases, a brute-force
 token-level block score, dense causal attention written separately, and
 invariants). Two parts stay "parity unpinned": real predictor boundaries and
-real row budgets (the trained weights do not exist here), so offsets and k
-are inputs.
+real row budgets (the trained weights do not exist here), so offsets, k and
+the token budgets are inputs. The row-budget rule itself is a reading of the
+pages (they name the budget but fix no formula); its pins check it against
+the top-k rule it reduces to and against closed forms.
 """
 from __future__ import annotations
 
@@ -127,6 +129,75 @@ def near_tie(S_row: np.ndarray, i: int, k: int, rel: float = 1e-5) -> bool:
         return False
     scale = float(np.max(np.abs(S_row[:i])))
     return tie_gap(S_row, i, k) < rel * scale
+
+
+# ---------------------------------------------------------------- a3': row budgets
+# README, "Predictor Checkpoints": static checkpoints use a fixed row budget,
+# dynamic ones a query-dependent row budget. gist.science technical summary,
+# "Significance and Claims" (Scalability): N_b is the token budget and the
+# per-layer cost is about O(L * N_b). The codewithpapers record names
+# recent-key-block and row-budget helpers but shows no code. Reading taken
+# (the pages fix no formula): a row keeps its diagonal chunk, the `recent`
+# chunks just before it, and then earlier chunks in rank order (score
+# descending, ties to the lower index) while the kept earlier tokens are
+# still fewer than the budget, at most k_max earlier chunks in all.
+def select_budget_row(S_row: np.ndarray, lens: np.ndarray, i: int, budget: int, recent: int,
+                      k_max: int) -> np.ndarray:
+    """Kept chunks of query chunk i under a token budget; ascending, i last.
+
+    lens[j] is the token length of chunk j. The recent window is the last
+    r = min(recent, i, k_max) chunks before i; ranked chunks are the j < i - r.
+    """
+    r = min(recent, i, k_max)
+    recent_js = list(range(i - r, i))
+    used = int(sum(int(lens[j]) for j in recent_js))
+    cand = np.arange(i - r)
+    order = cand[np.argsort(-S_row[: i - r], kind="stable")]
+    taken = []
+    for j in order:
+        if len(taken) + r >= k_max or used >= budget:
+            break
+        taken.append(int(j))
+        used += int(lens[j])
+    keep = sorted(taken) + recent_js
+    return np.array(keep + [i], dtype=np.int64)
+
+
+def select_budget(S: np.ndarray, off: np.ndarray, n_chunks: np.ndarray, budget, recent: int, k_max: int):
+    """sel[b][hq][i] under a token budget: an int for every row, or an int
+    array [B, Hq, Nmax] of per-row budgets."""
+    B, Hq = S.shape[:2]
+    out = []
+    for b in range(B):
+        n = int(n_chunks[b])
+        lens = np.diff(off[b][: n + 1])
+        rows_b = []
+        for hq in range(Hq):
+            rows_b.append([select_budget_row(S[b, hq, i], lens, i,
+                                             int(budget if np.isscalar(budget) else budget[b, hq, i]),
+                                             recent, k_max) for i in range(n)])
+        out.append(rows_b)
+    return out
+
+
+def budget_near_tie(S_row: np.ndarray, lens: np.ndarray, i: int, budget: int, recent: int, k_max: int,
+                    rel: float = 1e-5) -> bool:
+    """The kept set can change under a swap of two ranked chunks whose scores
+    differ by less than rel * max_j |S[i, j]| anywhere in the ranked prefix
+    the rule inspects (its taken chunks and the next one)."""
+    r = min(recent, i, k_max)
+    c = i - r
+    if c < 2:
+        return False
+    kept = select_budget_row(S_row, lens, i, budget, recent, k_max)
+    t = len(kept) - 1 - r                # ranked chunks taken
+    last = min(t + 1, c)                 # ranks 0 .. last-1 decide the set
+    srt = np.sort(S_row[:c])[::-1]
+    scale = float(np.max(np.abs(S_row[:i])))
+    gaps = srt[: last - 1] - srt[1:last] if last >= 2 else np.array([])
+    if last < c:                         # the boundary pair
+        gaps = np.append(gaps, srt[last - 1] - srt[last])
+    return bool(gaps.size and gaps.min() < rel * scale)
 
 
 # ---------------------------------------------------------------- a4: CSR

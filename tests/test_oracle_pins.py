@@ -306,3 +306,103 @@ def test_frozen_k_for_8k_workload():
     off, nc, S = freeze_k.pooled_scores(w, I)
     assert freeze_k.density_for_k(S, off, nc, w.k, w.L) >= w.target_density
     assert freeze_k.density_for_k(S, off, nc, w.k - 1, w.L) < w.target_density
+
+
+# ---------------------------------------------------------------- row budgets
+def test_budget_hand_cases():
+    g = json.load(open(os.path.join(GOLDEN, "budget_hand_cases.json")))
+    S = np.array(g["row"]["S"])
+    lens = np.array(g["row"]["lens"])
+    i = g["row"]["i"]
+    for c in g["cases"]:
+        got = dhsa.select_budget_row(S, lens, i, c["budget"], c["recent"], c["k_max"])
+        assert got.tolist() == c["expect"], c
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_budget_reduces_to_topk(seed):
+    # a budget no row can fill, no window: the top-k_max rule (pinned above
+    # against the brute-force token-level block score)
+    rng = np.random.default_rng(seed)
+    n = 40
+    lens = rng.integers(1, 50, n)
+    for i in range(n):
+        S = rng.standard_normal(n)
+        S[rng.integers(0, n, 5)] = 0.25          # a few exact ties
+        for k_max in (0, 1, 3, 7, 50):
+            got = dhsa.select_budget_row(S, lens, i, 10 ** 9, 0, k_max)
+            assert got.tolist() == dhsa.select_row(S, i, k_max).tolist()
+
+
+def test_budget_uniform_lengths_is_topk_of_budget_over_length():
+    rng = np.random.default_rng(7)
+    n, ln = 30, 16
+    lens = np.full(n, ln)
+    for i in range(n):
+        S = rng.standard_normal(n)
+        for m in range(0, 8):
+            for extra in (0, 1, ln - 1):          # budgets m*ln - extra .. round up to m chunks
+                budget = m * ln - extra if m > 0 else 0
+                want = dhsa.select_row(S, i, m)
+                got = dhsa.select_budget_row(S, lens, i, budget, 0, 100)
+                assert got.tolist() == want.tolist(), (i, m, extra)
+
+
+def test_budget_zero_keeps_recent_window_only():
+    S = np.linspace(1.0, -1.0, 20)
+    lens = np.arange(1, 21)
+    for i in range(20):
+        for r in (0, 1, 3, 25):
+            got = dhsa.select_budget_row(S, lens, i, 0, r, 100)
+            assert got.tolist() == list(range(max(0, i - r), i)) + [i]
+
+
+def test_budget_invariants_random():
+    rng = np.random.default_rng(11)
+    n = 60
+    for trial in range(30):
+        lens = rng.integers(1, 80, n)
+        S = rng.standard_normal(n)
+        i = int(rng.integers(0, n))
+        r = int(rng.integers(0, 5))
+        k_max = int(rng.integers(0, 20))
+        prev = None
+        for budget in (0, 10, 50, 200, 800, 10 ** 6):
+            kept = dhsa.select_budget_row(S, lens, i, budget, r, k_max)
+            assert kept[-1] == i and np.all(np.diff(kept) > 0)
+            earlier = kept[:-1]
+            assert len(earlier) <= max(k_max, 0)
+            rr = min(r, i, k_max)
+            assert set(range(i - rr, i)) <= set(earlier.tolist())
+            ranked = [j for j in earlier if j < i - rr]
+            used = int(lens[i - rr:i].sum()) + int(sum(int(lens[j]) for j in ranked))
+            # the ranked picks are a prefix of the (score desc, index asc) order
+            order = np.argsort(-S[: i - rr], kind="stable")
+            t = len(ranked)
+            assert sorted(order[:t].tolist()) == ranked
+            # stopping rule: below the budget before the last pick; when the fill
+            # stopped early, the budget was met or the cap reached
+            if t:
+                assert used - int(lens[order[t - 1]]) < budget
+            if t < i - rr and len(earlier) < k_max:
+                assert used >= budget
+            if prev is not None:                     # monotone in the budget
+                assert set(prev.tolist()) <= set(kept.tolist())
+            prev = kept
+
+
+def test_budget_vector_matches_per_row_scalar():
+    rng = np.random.default_rng(3)
+    B, Hq, n = 2, 3, 12
+    off = np.zeros((B, n + 1), dtype=np.int64)
+    for b in range(B):
+        off[b, 1:] = np.cumsum(rng.integers(1, 9, n))
+    S = rng.standard_normal((B, Hq, n, n))
+    budgets = rng.integers(0, 30, (B, Hq, n))
+    sel = dhsa.select_budget(S, off, np.array([n, n]), budgets, 1, 5)
+    for b in range(B):
+        lens = np.diff(off[b])
+        for hq in range(Hq):
+            for i in range(n):
+                want = dhsa.select_budget_row(S[b, hq, i], lens, i, int(budgets[b, hq, i]), 1, 5)
+                assert sel[b][hq][i].tolist() == want.tolist()
