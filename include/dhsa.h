@@ -129,6 +129,38 @@ int dhsa_chunk_score_topk(const float* Qp, const float* Kp, int B, int Hq, int H
                           size_t workspace_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * 2'. Chunk similarity and causal selection under a token budget per row.
+ *    Sources: README, "Predictor Checkpoints" (static checkpoints use a fixed
+ *    row budget, dynamic ones a query-dependent row budget); gist.science
+ *    technical summary, "Significance and Claims" (N_b is the token budget,
+ *    cost about O(L * N_b)). The pages give no formula; the rule implemented
+ *    (and restated by the test oracle) is:
+ *
+ *    For each row (b, hq, i < n_chunks[b]), with n_j = off[b][j+1] - off[b][j]:
+ *      r      = min(recent, i, k_max)   -- the chunks i-r .. i-1 are always kept
+ *      N_b    = budgets ? budgets[b,hq,i] : budget
+ *      ranked = the chunks j < i - r by (S descending, j ascending), S as in 2.
+ *      walk the ranked chunks in order, keeping each while fewer than
+ *      k_max - r have been kept and the kept earlier tokens (recent window
+ *      included) are still fewer than N_b;
+ *      sel[b,hq,i, ...] = kept ranked chunks, then the window, then i
+ *      (ascending), the rest -1; n_sel = their count (<= k_max + 1).
+ *    Rows i >= n_chunks[b] get n_sel = 0 and are filled with -1.
+ *
+ *    off      int32 [B, Nmax+1] as in 1.;  budgets int32 [B, Hq, Nmax] or NULL
+ *    budget   >= 0 (used when budgets is NULL);  recent >= 0
+ *    k_max    0 .. dhsa_budget_max_chunks() (UNSUPPORTED above it)
+ *    sel      int32 [B, Hq, Nmax, dhsa_sel_stride(k_max, Nmax)];  n_sel as in 2.
+ *    workspace: dhsa_score_topk_workspace_size(B, Hq, Nmax) bytes.
+ *    The CSR of 3. is then built with k = k_max.
+ * ------------------------------------------------------------------------- */
+int dhsa_budget_max_chunks(void);
+int dhsa_chunk_score_select_budget(const float* Qp, const float* Kp, int B, int Hq, int Hkv, int Nmax,
+                                   const int32_t* off, const int32_t* n_chunks, int budget,
+                                   const int32_t* budgets, int recent, int k_max, int32_t* sel, int32_t* n_sel,
+                                   void* workspace, size_t workspace_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
  * 3. Upsampling to the token keep-set, stored as a block CSR.
  *    Source: OpenReview abstract (chunk scores are upsampled to the token
  *    level to decide which token interactions are kept); gist.science

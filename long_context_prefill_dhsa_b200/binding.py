@@ -49,6 +49,8 @@ _SIGNATURES = {
     "dhsa_sel_stride": (_I, [_I, _I]),
     "dhsa_score_topk_workspace_size": (_SZ, [_I, _I, _I]),
     "dhsa_chunk_score_topk": (_I, [_P, _P, _I, _I, _I, _I, _P, _I, _P, _P, _P, _SZ, _P]),
+    "dhsa_budget_max_chunks": (_I, []),
+    "dhsa_chunk_score_select_budget": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, _I, _P, _I, _I, _P, _P, _P, _SZ, _P]),
     "dhsa_csr_nnz_upper": (_SZ, [_I, _I, _I, _I]),
     "dhsa_build_block_csr": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P]),
     "dhsa_sparse_attn_workspace_size": (_SZ, [_I, _I, _I, _I]),
@@ -171,6 +173,42 @@ def chunk_score_topk(Qp: torch.Tensor, Kp: torch.Tensor, n_chunks: torch.Tensor,
     return sel, n_sel
 
 
+def chunk_score_select_budget(Qp: torch.Tensor, Kp: torch.Tensor, off: torch.Tensor, n_chunks: torch.Tensor,
+                              budget, recent: int, k_max: int, sel: Optional[torch.Tensor] = None,
+                              n_sel: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None):
+    """Selection under a token budget per row (see include/dhsa.h, 2').
+
+    `budget` is an int (every row) or an int32 CUDA tensor [B, Hq, Nmax] of
+    per-row budgets. Returns sel [B,Hq,Nmax,stride(k_max)] and n_sel."""
+    B, Hq, nmax, d = Qp.shape
+    Hkv = Kp.shape[1]
+    _need(Qp, torch.float32, None, "Qp")
+    _need(Kp, torch.float32, (B, Hkv, nmax, d), "Kp")
+    _need(off, torch.int32, (B, nmax + 1), "off")
+    _need(n_chunks, torch.int32, (B,), "n_chunks")
+    budgets = None
+    if isinstance(budget, torch.Tensor):
+        _need(budget, torch.int32, (B, Hq, nmax), "budget")
+        budgets, budget = budget, 0
+    lib = load()
+    stride = lib.dhsa_sel_stride(k_max, nmax)
+    if sel is None:
+        sel = torch.empty((B, Hq, nmax, stride), dtype=torch.int32, device=Qp.device)
+    if n_sel is None:
+        n_sel = torch.empty((B, Hq, nmax), dtype=torch.int32, device=Qp.device)
+    _need(sel, torch.int32, (B, Hq, nmax, stride), "sel")
+    _need(n_sel, torch.int32, (B, Hq, nmax), "n_sel")
+    ws_bytes = lib.dhsa_score_topk_workspace_size(B, Hq, nmax)
+    if ws_bytes and workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=Qp.device)
+    ws_ptr = _ptr(workspace) if ws_bytes else None
+    ws_len = workspace.numel() * workspace.element_size() if (ws_bytes and workspace is not None) else 0
+    _check(lib.dhsa_chunk_score_select_budget(_ptr(Qp), _ptr(Kp), B, Hq, Hkv, nmax, _ptr(off), _ptr(n_chunks),
+                                              int(budget), _ptr(budgets), recent, k_max, _ptr(sel), _ptr(n_sel),
+                                              ws_ptr, ws_len, _stream_ptr()), "dhsa_chunk_score_select_budget")
+    return sel, n_sel
+
+
 def build_block_csr(sel: torch.Tensor, n_sel: torch.Tensor, k: int, off: torch.Tensor, n_chunks: torch.Tensor,
                     row_ptr=None, col_idx=None, cost=None, want_cost: bool = True):
     B, Hq, nmax, stride = sel.shape
@@ -239,14 +277,18 @@ def sparse_attn_fwd_noalloc(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, o
 class DHSAPrefill:
     """The five calls of one DHSA prefill layer with buffers allocated once.
 
-    run(Q, K, V) does pool(Q), pool(K), score + top-k, CSR build and sparse
-    attention on the current stream and returns O (bf16, like Q).
+    run(Q, K, V) does pool(Q), pool(K), score + selection, CSR build and
+    sparse attention on the current stream and returns O (bf16, like Q).
+    Selection is the top-k rule, or, when `budget` is given (an int, or an
+    int32 tensor [B, Hq, Nmax] of per-row budgets), the token-budget rule with
+    a window of `recent` chunks and at most k earlier chunks per row.
     """
 
     def __init__(self, B: int, Hq: int, Hkv: int, L: int, off: torch.Tensor, n_chunks: torch.Tensor, k: int,
-                 device="cuda", softmax_scale: Optional[float] = None):
+                 device="cuda", softmax_scale: Optional[float] = None, budget=None, recent: int = 0):
         lib = load()
         self.B, self.Hq, self.Hkv, self.L, self.k = B, Hq, Hkv, L, k
+        self.budget, self.recent = budget, recent
         self.off, self.n_chunks = off, n_chunks
         self.nmax = off.shape[1] - 1
         nmax = self.nmax
@@ -269,8 +311,12 @@ class DHSAPrefill:
     def routing(self, Q, K):
         chunk_pool(Q, self.off, self.n_chunks, out=self.Qp)
         chunk_pool(K, self.off, self.n_chunks, out=self.Kp)
-        chunk_score_topk(self.Qp, self.Kp, self.n_chunks, self.k, sel=self.sel, n_sel=self.n_sel,
-                         workspace=self.ws_topk)
+        if self.budget is None:
+            chunk_score_topk(self.Qp, self.Kp, self.n_chunks, self.k, sel=self.sel, n_sel=self.n_sel,
+                             workspace=self.ws_topk)
+        else:
+            chunk_score_select_budget(self.Qp, self.Kp, self.off, self.n_chunks, self.budget, self.recent, self.k,
+                                      sel=self.sel, n_sel=self.n_sel, workspace=self.ws_topk)
         build_block_csr(self.sel, self.n_sel, self.k, self.off, self.n_chunks, row_ptr=self.row_ptr,
                         col_idx=self.col_idx, cost=self.cost)
 

@@ -14,6 +14,10 @@ int score_topk_stride(int k, int Nmax);
 size_t score_topk_ws_bytes(int B, int Hq, int Nmax);
 int launch_score_topk(const float* Qp, const float* Kp, int B, int Hq, int Hkv, int Nmax, const int32_t* n_chunks,
                       int k, int32_t* sel, int32_t* n_sel, void* ws, cudaStream_t stream);
+int score_budget_max_chunks();
+int launch_score_budget(const float* Qp, const float* Kp, int B, int Hq, int Hkv, int Nmax, const int32_t* off,
+                        const int32_t* n_chunks, int budget, const int32_t* budgets, int recent, int k_max,
+                        int32_t* sel, int32_t* n_sel, void* ws, cudaStream_t stream);
 int launch_build_csr(const int32_t* sel, const int32_t* n_sel, int B, int Hq, int Nmax, int k, const int32_t* off,
                      const int32_t* n_chunks, int32_t* row_ptr, int32_t* col_idx, int64_t* cost,
                      unsigned int* status, cudaStream_t stream);
@@ -158,6 +162,24 @@ int dhsa_chunk_score_topk(const float* Qp, const float* Kp, int B, int Hq, int H
   if (st != DHSA_OK) return st;
   return launch_score_topk(Qp, Kp, B, Hq, Hkv, Nmax, n_chunks, k, sel, n_sel, need ? workspace : nullptr,
                            static_cast<cudaStream_t>(stream));
+}
+
+int dhsa_budget_max_chunks(void) { return score_budget_max_chunks(); }
+
+int dhsa_chunk_score_select_budget(const float* Qp, const float* Kp, int B, int Hq, int Hkv, int Nmax,
+                                   const int32_t* off, const int32_t* n_chunks, int budget,
+                                   const int32_t* budgets, int recent, int k_max, int32_t* sel, int32_t* n_sel,
+                                   void* workspace, size_t workspace_bytes, void* stream) {
+  if (!Qp || !Kp || !off || !n_chunks || !sel || !n_sel) return DHSA_ERR_INVALID_ARG;
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Nmax <= 0 || Hq % Hkv != 0) return DHSA_ERR_INVALID_ARG;
+  if (k_max < 0 || recent < 0 || (!budgets && budget < 0)) return DHSA_ERR_INVALID_ARG;
+  if (k_max > score_budget_max_chunks()) return DHSA_ERR_UNSUPPORTED;
+  const size_t need = score_topk_ws_bytes(B, Hq, Nmax);
+  if (need && (!workspace || workspace_bytes < need || !aligned16(workspace))) return DHSA_ERR_WORKSPACE;
+  int st = check_device_sm100();
+  if (st != DHSA_OK) return st;
+  return launch_score_budget(Qp, Kp, B, Hq, Hkv, Nmax, off, n_chunks, budget, budgets, recent, k_max, sel, n_sel,
+                             need ? workspace : nullptr, static_cast<cudaStream_t>(stream));
 }
 
 size_t dhsa_csr_nnz_upper(int B, int Hq, int Nmax, int k) {

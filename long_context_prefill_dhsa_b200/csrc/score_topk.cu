@@ -34,6 +34,7 @@ constexpr int kKsStride = kHeadDim + 4;
 constexpr size_t kWsCap = size_t(256) << 20;   // scores of one head batch
 constexpr double kU = 5.9604644775390625e-08;   // 2^-24
 constexpr double kGamma = 128.0 * kU / (1.0 - 128.0 * kU);
+constexpr int kBudgetCap = 256;   // a budget row keeps at most kBudgetCap - 1 earlier chunks
 
 __device__ __forceinline__ unsigned order_key32(float s) {
   const unsigned u = __float_as_uint(s);
@@ -147,6 +148,184 @@ __device__ __forceinline__ bool ranks_above(double sa, int ja, double sb, int jb
   return sa > sb || (sa == sb && ja < jb);
 }
 
+// The exact top-m of candidates j < c of one row, m < c, as a cut: scores
+// above hi are in, below lo are out, and a band score is in iff it does not
+// rank below (cutE, cutJ) (or the whole band is in). Executed by one warp;
+// `hist` is that warp's 256-int shared scratch.
+struct Cut {
+  double lo, hi, cutE;
+  int cutJ;
+  bool all_band;
+};
+
+__device__ Cut topm_cut(const float* __restrict__ row, int c, int m, int* hist, const float* __restrict__ qrow,
+                        const float* __restrict__ Kp, long long kv_row0, const float* __restrict__ kn) {
+  const int lane = threadIdx.x & 31;
+  const unsigned full = 0xffffffffu;
+  // --- radix select of the m-th largest fp32 key
+  unsigned prefix = 0, mask = 0;
+  int need = m;
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int q = lane; q < 256; q += 32) hist[q] = 0;
+    __syncwarp();
+    for (int j = lane; j < c; j += 32) {
+      const unsigned kk = order_key32(row[j]);
+      if ((kk & mask) == prefix) atomicAdd(&hist[(kk >> shift) & 255], 1);
+    }
+    __syncwarp();
+    int cq[8], lsum = 0;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      cq[q] = hist[255 - 8 * lane - q];
+      lsum += cq[q];
+    }
+    int incl = lsum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(full, incl, o);
+      if (lane >= o) incl += t;
+    }
+    const int excl = incl - lsum;
+    const unsigned ball = __ballot_sync(full, excl < need && need <= incl);
+    const int src = __ffs(ball) - 1;
+    int digit = 0, above = 0;
+    if (lane == src) {
+      int run = excl;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        if (run + cq[q] >= need) {
+          digit = 255 - 8 * lane - q;
+          above = run;
+          break;
+        }
+        run += cq[q];
+      }
+    }
+    digit = __shfl_sync(full, digit, src);
+    above = __shfl_sync(full, above, src);
+    prefix |= (unsigned)digit << shift;
+    mask |= 0xFFu << shift;
+    need -= above;
+    __syncwarp();
+  }
+  const unsigned tu = (prefix & 0x80000000u) ? (prefix & 0x7fffffffu) : ~prefix;
+  const double T = (double)__uint_as_float(tu);
+  // --- rounding band
+  const float4 qv = reinterpret_cast<const float4*>(qrow)[lane];
+  double qq = (double)qv.x * qv.x + (double)qv.y * qv.y + (double)qv.z * qv.z + (double)qv.w * qv.w;
+  float kmax = 0.f;
+  for (int j = lane; j < c; j += 32) kmax = fmaxf(kmax, kn[kv_row0 + j]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    qq += __shfl_xor_sync(full, qq, o);
+    kmax = fmaxf(kmax, __shfl_xor_sync(full, kmax, o));
+  }
+  const double D = 2.0 * kGamma * sqrt(qq) * (1.0 + 1e-6) * (double)kmax;
+  Cut cut;
+  cut.lo = T - D;
+  cut.hi = T + D;
+  cut.cutE = -INFINITY;
+  cut.cutJ = 0x7fffffff;
+  int a = 0, nc = 0;
+  for (int j = lane; j < c; j += 32) {
+    const double s = (double)row[j];
+    a += s > cut.hi;
+    nc += (s >= cut.lo && s <= cut.hi);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    a += __shfl_xor_sync(full, a, o);
+    nc += __shfl_xor_sync(full, nc, o);
+  }
+  const int r = m - a;              // 1 <= r <= nc
+  // --- exact cut (E*, j*) among the band: the r-th by (exact desc, j asc)
+  cut.all_band = (r >= nc);
+  if (cut.all_band) return cut;
+  if (nc <= 32) {
+    // compact the band into lanes 0..nc-1 (through the free histogram area),
+    // score exactly, bitonic sort best-first
+    int base = 0;
+    for (int j0 = 0; j0 < c; j0 += 32) {
+      const int j = j0 + lane;
+      bool inb = false;
+      if (j < c) {
+        const double s = (double)row[j];
+        inb = s >= cut.lo && s <= cut.hi;
+      }
+      const unsigned bb = __ballot_sync(full, inb);
+      if (inb) hist[base + __popc(bb & lanemask_lt())] = j;
+      base += __popc(bb);
+    }
+    __syncwarp();
+    const int my_j = lane < nc ? hist[lane] : -1;
+    __syncwarp();
+    double my_e = -INFINITY;
+    int my_key_j = 0x7fffffff;
+    if (my_j >= 0) {
+      my_e = exact_score(qrow, Kp + (kv_row0 + my_j) * kHeadDim);
+      my_key_j = my_j;
+    }
+#pragma unroll
+    for (int size = 2; size <= 32; size <<= 1) {
+#pragma unroll
+      for (int stride2 = size >> 1; stride2 > 0; stride2 >>= 1) {
+        const double oe = __shfl_xor_sync(full, my_e, stride2);
+        const int oj = __shfl_xor_sync(full, my_key_j, stride2);
+        const bool up = ((lane & size) == 0);          // this block sorts best-first
+        const bool lower = ((lane & stride2) == 0);
+        const bool mine_above = ranks_above(my_e, my_key_j, oe, oj);
+        const bool keep_mine = (lower == up) ? mine_above : !mine_above;
+        if (!keep_mine) {
+          my_e = oe;
+          my_key_j = oj;
+        }
+      }
+    }
+    cut.cutE = __shfl_sync(full, my_e, r - 1);
+    cut.cutJ = __shfl_sync(full, my_key_j, r - 1);
+  } else {
+    // many candidates (heavy ties): r rounds of "best below the previous pick"
+    double pe = INFINITY;
+    int pj = -1;
+    for (int t = 0; t < r; ++t) {
+      double be = -INFINITY;
+      int bj = 0x7fffffff;
+      for (int j = lane; j < c; j += 32) {
+        const double s = (double)row[j];
+        if (s < cut.lo || s > cut.hi) continue;
+        const double e = exact_score(qrow, Kp + (kv_row0 + j) * kHeadDim);
+        if (ranks_above(pe, pj, e, j) && ranks_above(e, j, be, bj)) {
+          be = e;
+          bj = j;
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const double oe = __shfl_xor_sync(full, be, o);
+        const int oj = __shfl_xor_sync(full, bj, o);
+        if (ranks_above(oe, oj, be, bj)) {
+          be = oe;
+          bj = oj;
+        }
+      }
+      pe = be;
+      pj = bj;
+    }
+    cut.cutE = pe;
+    cut.cutJ = pj;
+  }
+  return cut;
+}
+
+// Is candidate j (fp32 score s) inside the exact top-m described by `cut`?
+__device__ __forceinline__ bool in_cut(const Cut& cut, float s32, int j, const float* __restrict__ qrow,
+                                       const float* __restrict__ Kp, long long kv_row0) {
+  const double s = (double)s32;
+  if (s > cut.hi) return true;
+  if (s < cut.lo) return false;
+  return cut.all_band || !ranks_above(cut.cutE, cut.cutJ, exact_score(qrow, Kp + (kv_row0 + j) * kHeadDim), j);
+}
+
 __global__ void __launch_bounds__(256) select_kernel(const float* __restrict__ Qp, const float* __restrict__ Kp,
                                                      const float* __restrict__ kn, int Hq, int G, int Nmax,
                                                      const int32_t* __restrict__ n_chunks, int k, int stride,
@@ -164,7 +343,6 @@ __global__ void __launch_bounds__(256) select_kernel(const float* __restrict__ Q
   const int b = (int)(bh / Hq), hq = (int)(bh % Hq);
   const int n = n_chunks[b];
   int32_t* out = sel + (bh * Nmax + i) * stride;
-  int* hist = hist_all[warp];
   int cnt = 0;
   if (i < n) {
     const int m = min(k, i);
@@ -173,174 +351,14 @@ __global__ void __launch_bounds__(256) select_kernel(const float* __restrict__ Q
       cnt = i;
     } else if (m > 0) {
       const float* row = ws + bhl * tri(Nmax) + tri(i);
-      // --- radix select of the m-th largest fp32 key
-      unsigned prefix = 0, mask = 0;
-      int need = m;
-      for (int shift = 24; shift >= 0; shift -= 8) {
-        for (int q = lane; q < 256; q += 32) hist[q] = 0;
-        __syncwarp();
-        for (int j = lane; j < i; j += 32) {
-          const unsigned kk = order_key32(row[j]);
-          if ((kk & mask) == prefix) atomicAdd(&hist[(kk >> shift) & 255], 1);
-        }
-        __syncwarp();
-        int c[8], lsum = 0;
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          c[q] = hist[255 - 8 * lane - q];
-          lsum += c[q];
-        }
-        int incl = lsum;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const int t = __shfl_up_sync(full, incl, o);
-          if (lane >= o) incl += t;
-        }
-        const int excl = incl - lsum;
-        const unsigned ball = __ballot_sync(full, excl < need && need <= incl);
-        const int src = __ffs(ball) - 1;
-        int digit = 0, above = 0;
-        if (lane == src) {
-          int run = excl;
-#pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            if (run + c[q] >= need) {
-              digit = 255 - 8 * lane - q;
-              above = run;
-              break;
-            }
-            run += c[q];
-          }
-        }
-        digit = __shfl_sync(full, digit, src);
-        above = __shfl_sync(full, above, src);
-        prefix |= (unsigned)digit << shift;
-        mask |= 0xFFu << shift;
-        need -= above;
-        __syncwarp();
-      }
-      const unsigned tu = (prefix & 0x80000000u) ? (prefix & 0x7fffffffu) : ~prefix;
-      const double T = (double)__uint_as_float(tu);
-      // --- rounding band
       const long long kv_row0 = ((long long)b * (Hq / G) + hq / G) * Nmax;
       const float* qrow = Qp + (bh * Nmax + i) * kHeadDim;
-      const float4 qv = reinterpret_cast<const float4*>(qrow)[lane];
-      double qq = (double)qv.x * qv.x + (double)qv.y * qv.y + (double)qv.z * qv.z + (double)qv.w * qv.w;
-      float kmax = 0.f;
-      for (int j = lane; j < i; j += 32) kmax = fmaxf(kmax, kn[kv_row0 + j]);
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        qq += __shfl_xor_sync(full, qq, o);
-        kmax = fmaxf(kmax, __shfl_xor_sync(full, kmax, o));
-      }
-      const double D = 2.0 * kGamma * sqrt(qq) * (1.0 + 1e-6) * (double)kmax;
-      const double lo = T - D, hi = T + D;
-      int a = 0, nc = 0;
-      for (int j = lane; j < i; j += 32) {
-        const double s = (double)row[j];
-        a += s > hi;
-        nc += (s >= lo && s <= hi);
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        a += __shfl_xor_sync(full, a, o);
-        nc += __shfl_xor_sync(full, nc, o);
-      }
-      const int r = m - a;              // 1 <= r <= nc
-      // --- exact cut (E*, j*) among the band: the r-th by (exact desc, j asc)
-      double cutE = -INFINITY;
-      int cutJ = 0x7fffffff;
-      bool take_all_band = (r >= nc);
-      if (!take_all_band) {
-        if (nc <= 32) {
-          // compact the band into lanes 0..nc-1 (through this warp's free
-          // histogram area), score exactly, bitonic sort best-first
-          int base = 0;
-          for (int j0 = 0; j0 < i; j0 += 32) {
-            const int j = j0 + lane;
-            bool inb = false;
-            if (j < i) {
-              const double s = (double)row[j];
-              inb = s >= lo && s <= hi;
-            }
-            const unsigned bb = __ballot_sync(full, inb);
-            if (inb) hist[base + __popc(bb & lanemask_lt())] = j;
-            base += __popc(bb);
-          }
-          __syncwarp();
-          const int my_j = lane < nc ? hist[lane] : -1;
-          __syncwarp();
-          double my_e = -INFINITY;
-          int my_key_j = 0x7fffffff;
-          if (my_j >= 0) {
-            my_e = exact_score(qrow, Kp + (kv_row0 + my_j) * kHeadDim);
-            my_key_j = my_j;
-          }
-          // bitonic sort of 32 (e, j) pairs, best first
-#pragma unroll
-          for (int size = 2; size <= 32; size <<= 1) {
-#pragma unroll
-            for (int stride2 = size >> 1; stride2 > 0; stride2 >>= 1) {
-              const double oe = __shfl_xor_sync(full, my_e, stride2);
-              const int oj = __shfl_xor_sync(full, my_key_j, stride2);
-              const bool up = ((lane & size) == 0);          // this block sorts best-first
-              const bool lower = ((lane & stride2) == 0);
-              const bool mine_above = ranks_above(my_e, my_key_j, oe, oj);
-              const bool keep_mine = (lower == up) ? mine_above : !mine_above;
-              if (!keep_mine) {
-                my_e = oe;
-                my_key_j = oj;
-              }
-            }
-          }
-          cutE = __shfl_sync(full, my_e, r - 1);
-          cutJ = __shfl_sync(full, my_key_j, r - 1);
-        } else {
-          // many candidates (heavy ties): r rounds of "best below the previous pick"
-          double pe = INFINITY;
-          int pj = -1;
-          for (int t = 0; t < r; ++t) {
-            double be = -INFINITY;
-            int bj = 0x7fffffff;
-            for (int j = lane; j < i; j += 32) {
-              const double s = (double)row[j];
-              if (s < lo || s > hi) continue;
-              const double e = exact_score(qrow, Kp + (kv_row0 + j) * kHeadDim);
-              if (ranks_above(pe, pj, e, j) && ranks_above(e, j, be, bj)) {
-                be = e;
-                bj = j;
-              }
-            }
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-              const double oe = __shfl_xor_sync(full, be, o);
-              const int oj = __shfl_xor_sync(full, bj, o);
-              if (ranks_above(oe, oj, be, bj)) {
-                be = oe;
-                bj = oj;
-              }
-            }
-            pe = be;
-            pj = bj;
-          }
-          cutE = pe;
-          cutJ = pj;
-        }
-      }
+      const Cut cut = topm_cut(row, i, m, hist_all[warp], qrow, Kp, kv_row0, kn);
       // --- output, ascending
       int written = 0;
       for (int j0 = 0; j0 < i; j0 += 32) {
         const int j = j0 + lane;
-        bool take = false;
-        if (j < i) {
-          const double s = (double)row[j];
-          if (s > hi) {
-            take = true;
-          } else if (s >= lo) {
-            take = take_all_band ||
-                   !ranks_above(cutE, cutJ, exact_score(qrow, Kp + (kv_row0 + j) * kHeadDim), j);
-          }
-        }
+        const bool take = j < i && in_cut(cut, row[j], j, qrow, Kp, kv_row0);
         const unsigned bt = __ballot_sync(full, take);
         const int pos = written + __popc(bt & lanemask_lt());
         if (take && pos < m) out[pos] = j;
@@ -348,6 +366,113 @@ __global__ void __launch_bounds__(256) select_kernel(const float* __restrict__ Q
       }
       cnt = written < m ? written : m;
     }
+    if (lane == 0) out[cnt] = i;
+    cnt += 1;
+  }
+  for (int q = cnt + lane; q < stride; q += 32) out[q] = -1;
+  if (lane == 0) n_sel[bh * Nmax + i] = cnt;
+}
+
+// ------------------------------------------------------------------ 3'. row budgets
+// README, "Predictor Checkpoints": fixed or query-dependent row budgets;
+// gist.science technical summary, "Significance and Claims": N_b is the token
+// budget. A row keeps its diagonal chunk, the r = min(recent, i, k_max)
+// chunks just before it, then earlier chunks j < i - r by (score desc,
+// index asc) while the kept earlier tokens are fewer than its budget, at
+// most k_max earlier chunks in all. Only the top m = min(k_max - r, i - r)
+// ranked candidates can be taken: their set comes from the same exact cut
+// as the top-k rule, then they are re-scored in fp64, ranked, and the
+// budget is applied along that order.
+__global__ void __launch_bounds__(256) budget_select_kernel(
+    const float* __restrict__ Qp, const float* __restrict__ Kp, const float* __restrict__ kn, int Hq, int G,
+    int Nmax, const int32_t* __restrict__ n_chunks, const int32_t* __restrict__ off, int budget,
+    const int32_t* __restrict__ budgets, int recent, int k_max, int stride, long long bh0, long long n_rows,
+    const float* __restrict__ ws, int32_t* __restrict__ sel, int32_t* __restrict__ n_sel) {
+  __shared__ int hist_all[8][256];
+  __shared__ int mj_all[8][kBudgetCap];      // members, ascending index
+  __shared__ double me_all[8][kBudgetCap];   // their exact scores
+  __shared__ int ml_all[8][kBudgetCap];      // chunk lengths by rank
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const unsigned full = 0xffffffffu;
+  const long long wr = (long long)blockIdx.x * 8 + warp;
+  if (wr >= n_rows) return;
+  const long long bhl = wr / Nmax;
+  const int i = (int)(wr % Nmax);
+  const long long bh = bh0 + bhl;
+  const int b = (int)(bh / Hq), hq = (int)(bh % Hq);
+  const int n = n_chunks[b];
+  int32_t* out = sel + (bh * Nmax + i) * stride;
+  int* hist = hist_all[warp];
+  int* mj = mj_all[warp];
+  double* me = me_all[warp];
+  int* ml = ml_all[warp];
+  int cnt = 0;
+  if (i < n) {
+    const int32_t* ob = off + (long long)b * (Nmax + 1);
+    const int r = min(min(recent, i), k_max);
+    const int c = i - r;                           // ranked candidates j < c
+    const int m = min(k_max - r, c);
+    const long long used0 = (long long)ob[i] - ob[i - r];
+    const long long bud = budgets ? (long long)budgets[bh * Nmax + i] : (long long)budget;
+    int t = 0;
+    if (m > 0 && used0 < bud) {
+      const float* row = ws + bhl * tri(Nmax) + tri(i);
+      const long long kv_row0 = ((long long)b * (Hq / G) + hq / G) * Nmax;
+      const float* qrow = Qp + (bh * Nmax + i) * kHeadDim;
+      const bool all = (m == c);
+      Cut cut{};
+      if (!all) cut = topm_cut(row, c, m, hist, qrow, Kp, kv_row0, kn);
+      // members of the top m, ascending index
+      int nm = 0;
+      for (int j0 = 0; j0 < c; j0 += 32) {
+        const int j = j0 + lane;
+        const bool take = j < c && (all || in_cut(cut, row[j], j, qrow, Kp, kv_row0));
+        const unsigned bt = __ballot_sync(full, take);
+        const int pos = nm + __popc(bt & lanemask_lt());
+        if (take && pos < m) mj[pos] = j;
+        nm += __popc(bt);
+      }
+      nm = min(nm, m);
+      __syncwarp();
+      for (int a = lane; a < nm; a += 32) me[a] = exact_score(qrow, Kp + (kv_row0 + mj[a]) * kHeadDim);
+      __syncwarp();
+      // rank of each member; lengths in rank order
+      for (int a = lane; a < nm; a += 32) {
+        const double ea = me[a];
+        const int ja = mj[a];
+        int rank = 0;
+        for (int q = 0; q < nm; ++q) rank += ranks_above(me[q], mj[q], ea, ja);
+        hist[a] = rank;
+        ml[rank] = ob[ja + 1] - ob[ja];
+      }
+      __syncwarp();
+      // ranks 0..t-1 are taken: those reached while the kept tokens are below the budget
+      long long run = used0;
+      for (int q0 = 0; q0 < nm; q0 += 32) {
+        const int q = q0 + lane;
+        const int v = q < nm ? ml[q] : 0;
+        int incl = v;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int u = __shfl_up_sync(full, incl, o);
+          if (lane >= o) incl += u;
+        }
+        t += __popc(__ballot_sync(full, q < nm && run + (incl - v) < bud));
+        run += __shfl_sync(full, incl, 31);
+      }
+      // taken members, ascending
+      int written = 0;
+      for (int a0 = 0; a0 < nm; a0 += 32) {
+        const int a = a0 + lane;
+        const bool take = a < nm && hist[a] < t;
+        const unsigned bt = __ballot_sync(full, take);
+        if (take) out[written + __popc(bt & lanemask_lt())] = mj[a];
+        written += __popc(bt);
+      }
+    }
+    cnt = t;
+    for (int q = lane; q < r; q += 32) out[cnt + q] = i - r + q;   // the recent window
+    cnt += r;
     if (lane == 0) out[cnt] = i;
     cnt += 1;
   }
@@ -399,6 +524,39 @@ int launch_score_topk(const float* Qp, const float* Kp, int B, int Hq, int Hkv, 
     const long long rows = nh * Nmax;
     select_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(Qp, Kp, kn, Hq, G, Nmax, n_chunks, k, stride, h0,
                                                                   rows, scores, sel, n_sel);
+    if ((st = launch_status()) != DHSA_OK) return st;
+  }
+  return DHSA_OK;
+}
+
+int score_budget_max_chunks() { return kBudgetCap - 1; }
+
+int launch_score_budget(const float* Qp, const float* Kp, int B, int Hq, int Hkv, int Nmax, const int32_t* off,
+                        const int32_t* n_chunks, int budget, const int32_t* budgets, int recent, int k_max,
+                        int32_t* sel, int32_t* n_sel, void* ws, cudaStream_t stream) {
+  const int G = Hq / Hkv;
+  const int stride = score_topk_stride(k_max, Nmax);
+  float* kn = reinterpret_cast<float*>(static_cast<char*>(ws) + 256);
+  const size_t kn_bytes = (sizeof(float) * (size_t)B * Hq * Nmax + 255) & ~size_t(255);
+  float* scores = reinterpret_cast<float*>(static_cast<char*>(ws) + 256 + kn_bytes);
+  const long long kv_rows = (long long)B * Hkv * Nmax;
+  key_norm_kernel<<<(unsigned)((kv_rows * 32 + 255) / 256), 256, 0, stream>>>(Kp, kv_rows, kn);
+  int st = launch_status();
+  if (st != DHSA_OK) return st;
+  const size_t smem = sizeof(float) * (TR * kHeadDim + TK * kKsStride);
+  cudaError_t e = cudaFuncSetAttribute(score_tile_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return cuda_status(e);
+  const int n_rb = (Nmax + TR - 1) / TR, n_kb = (Nmax + TK - 1) / TK;
+  const long long total = (long long)B * Hq, hb = heads_per_batch(B, Hq, Nmax);
+  for (long long h0 = 0; h0 < total; h0 += hb) {
+    const long long nh = (total - h0 < hb) ? total - h0 : hb;
+    dim3 grid((unsigned)(n_rb * n_kb), (unsigned)nh);
+    score_tile_kernel<<<grid, 256, smem, stream>>>(Qp, Kp, Hq, G, Nmax, n_chunks, h0, n_rb, n_kb, scores);
+    if ((st = launch_status()) != DHSA_OK) return st;
+    const long long rows = nh * Nmax;
+    budget_select_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(
+        Qp, Kp, kn, Hq, G, Nmax, n_chunks, off, budget, budgets, recent, k_max, stride, h0, rows, scores, sel,
+        n_sel);
     if ((st = launch_status()) != DHSA_OK) return st;
   }
   return DHSA_OK;

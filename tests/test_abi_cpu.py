@@ -69,3 +69,18 @@ def test_invalid_arguments_rejected_on_host(lib):
     args[7] = 128
     args[5] = 3      # Hq % Hkv != 0
     assert lib.dhsa_sparse_attn_fwd(*args, ctypes.c_float(0.1), FAKE, FAKE, big, None) == INV
+
+
+def test_budget_selection_arguments_rejected_on_host(lib):
+    INV, UNS, WS = 1, 2, 5
+    cap = lib.dhsa_budget_max_chunks()
+    assert cap >= 64
+    f = lib.dhsa_chunk_score_select_budget
+    #      Qp    Kp    B  Hq Hkv Nmax off   n_ch  budget budgets recent k_max sel   n_sel ws  bytes stream
+    assert f(FAKE, FAKE, 1, 4, 2, 8, FAKE, FAKE, 100, None, 0, cap + 1, FAKE, FAKE, FAKE, 1 << 30, None) == UNS
+    assert f(FAKE, FAKE, 1, 4, 2, 8, FAKE, FAKE, -1, None, 0, 4, FAKE, FAKE, FAKE, 1 << 30, None) == INV
+    assert f(FAKE, FAKE, 1, 4, 2, 8, FAKE, FAKE, 100, None, -1, 4, FAKE, FAKE, FAKE, 1 << 30, None) == INV
+    assert f(FAKE, FAKE, 1, 4, 2, 8, FAKE, FAKE, 100, None, 0, -1, FAKE, FAKE, FAKE, 1 << 30, None) == INV
+    assert f(FAKE, FAKE, 1, 4, 2, 8, None, FAKE, 100, None, 0, 4, FAKE, FAKE, FAKE, 1 << 30, None) == INV
+    assert f(FAKE, FAKE, 1, 3, 2, 8, FAKE, FAKE, 100, None, 0, 4, FAKE, FAKE, FAKE, 1 << 30, None) == INV
+    assert f(FAKE, FAKE, 1, 4, 2, 8, FAKE, FAKE, 100, None, 0, 4, FAKE, FAKE, None, 0, None) == WS
