@@ -52,7 +52,29 @@ def parse():
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    # selection rule: top-k (default), or a token budget per row with a recent
+    # window and a chunk cap; --budget-spread gives every row its own seeded
+    # budget, uniform in budget * [1 - spread, 1 + spread] (query-dependent budgets)
+    ap.add_argument("--budget", type=int, default=None)
+    ap.add_argument("--recent", type=int, default=0)
+    ap.add_argument("--kmax", type=int, default=None)
+    ap.add_argument("--budget-spread", type=float, default=0.0)
     return ap.parse_args()
+
+
+def selection_rule(args, w, nmax):
+    """(k passed to the layer, budget argument, recent, description) for the CLI options."""
+    if args.budget is None:
+        return w.k, None, 0, {"rule": "top-k", "k": w.k}
+    k_max = args.kmax if args.kmax is not None else 4 * w.k
+    desc = {"rule": "token budget", "budget": args.budget, "recent": args.recent, "k_max": k_max}
+    if args.budget_spread > 0:
+        rng = np.random.default_rng(1234)
+        lo, hi = args.budget * (1 - args.budget_spread), args.budget * (1 + args.budget_spread)
+        vec = rng.integers(int(lo), int(hi) + 1, (w.B, w.Hq, nmax)).astype(np.int32)
+        desc["budget_spread"] = args.budget_spread
+        return k_max, vec, args.recent, desc
+    return k_max, args.budget, args.recent, desc
 
 
 def attn_traffic(workload_name):
@@ -191,7 +213,7 @@ def attn_bytes(w):
 
 
 # ----------------------------------------------------------------- oracle (CPU) leg
-def cpu_oracle_sample(d, w, seconds):
+def cpu_oracle_sample(d, w, seconds, rule=None):
     """Time the CPU oracle on a bounded sample of the layer and extrapolate
     to ms per layer. Sample: pooling of one query head + its kv head, the
     chunk scores/selection of that head, and the attention of as many of its
@@ -206,7 +228,11 @@ def cpu_oracle_sample(d, w, seconds):
     t_pool = time.perf_counter() - t0
     t0 = time.perf_counter()
     S = ora.chunk_scores(Qp, Kp, nc)
-    sel = ora.select(S, nc, w.k)
+    if rule is None or rule[1] is None:
+        sel = ora.select(S, nc, w.k)
+    else:
+        k_max, bud, recent = rule[0], rule[1], rule[2]
+        sel = ora.select_budget(S, off, nc, bud if np.isscalar(bud) else bud[:, :1], recent, k_max)
     t_route = time.perf_counter() - t0
     Q = ora.bf16_to_f64(d["Q"][0, 0]).astype(np.float32)
     K = ora.bf16_to_f64(d["K"][0, 0]).astype(np.float32)
@@ -225,7 +251,7 @@ def cpu_oracle_sample(d, w, seconds):
     kv_frac = w.Hkv / w.Hq
     est = (t_pool * (1 + kv_frac) / 2 * heads + t_route * heads + t_attn * (n / done) * heads)
     return {"value": est * 1e3, "unit": "ms", "cores": cores, "kind": "oracle",
-            "sample": (f"oracle on (b=0, hq=0): pooling of Q and K, all {n} score/top-k rows, attention of "
+            "sample": (f"oracle on (b=0, hq=0): pooling of Q and K, all {n} score/selection rows, attention of "
                        f"{done}/{n} query chunks; extrapolated x{heads} heads"
                        f"{' x' + str(round(n / done, 2)) + ' chunks' if done < n else ''}")}
 
@@ -238,12 +264,14 @@ def run_reference(args):
     from long_context_prefill_dhsa_b200 import inputs as I
     w = I.WORKLOADS[args.workload]
     d = I.make_inputs(w)
+    k_sel, bud, recent, sel_desc = selection_rule(args, w, d["off"].shape[1] - 1)
+    rule = (k_sel, bud, recent)
     for _ in range(args.warmup):
-        cpu_oracle_sample(d, w, min(2.0, args.cpu_seconds))
+        cpu_oracle_sample(d, w, min(2.0, args.cpu_seconds), rule)
     vals = []
     res = None
     for _ in range(args.steps):
-        res = cpu_oracle_sample(d, w, args.cpu_seconds / max(1, args.steps))
+        res = cpu_oracle_sample(d, w, args.cpu_seconds / max(1, args.steps), rule)
         vals.append(res["value"])
     v = statistics.median(vals)
     res["value"] = v
@@ -252,7 +280,7 @@ def run_reference(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": v, "higher_is_better": False,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "L": w.L, "k": w.k,
-                   "chunk_len": f"{w.length_kind}[{w.length_lo},{w.length_hi}]"},
+                   "selection": sel_desc, "chunk_len": f"{w.length_kind}[{w.length_lo},{w.length_hi}]"},
         "cpu_baseline": res, "e2e": {"value": v, "unit": "ms", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }), flush=True)
 
@@ -284,7 +312,9 @@ def main():
     host_nc = torch.from_numpy(d["n_chunks"]).pin_memory()
     Q, K, V = (host[x].to(dev) for x in "QKV")
     off, nc = host_off.to(dev), host_nc.to(dev)
-    layer = binding.DHSAPrefill(w.B, w.Hq, w.Hkv, w.L, off, nc, w.k, device=dev)
+    k_sel, bud, recent, sel_desc = selection_rule(args, w, d["off"].shape[1] - 1)
+    bud_arg = torch.from_numpy(bud).to(dev) if isinstance(bud, np.ndarray) else bud
+    layer = binding.DHSAPrefill(w.B, w.Hq, w.Hkv, w.L, off, nc, k_sel, device=dev, budget=bud_arg, recent=recent)
     stream = torch.cuda.current_stream()
 
     ev = lambda: torch.cuda.Event(enable_timing=True)
@@ -330,7 +360,7 @@ def main():
     flop = 4.0 * 128 * pairs
     hbm_peak, tc_peak, peak_kind = peaks()
     attn_tflops = flop / (attn_ms * 1e-3) / 1e12
-    rbytes = routing_bytes(w, nmax, w.k)
+    rbytes = routing_bytes(w, nmax, k_sel)
     traffic, traffic_src = attn_traffic(w.name)
 
     # end to end through the public API with host buffers (pinned), on this rank
@@ -394,7 +424,7 @@ def main():
 
     cpu = None
     if not args.no_cpu and rank == 0 and world == 1:
-        cpu = cpu_oracle_sample(d, w, args.cpu_seconds)
+        cpu = cpu_oracle_sample(d, w, args.cpu_seconds, (k_sel, bud, recent))
 
     if rank == 0:
         line = {
@@ -403,7 +433,8 @@ def main():
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": False, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "L": w.L, "head_dim": 128,
-                       "k": w.k, "chunk_len": f"{w.length_kind}[{w.length_lo},{w.length_hi}]", "n_chunks": nmax,
+                       "k": w.k, "selection": sel_desc,
+                       "chunk_len": f"{w.length_kind}[{w.length_lo},{w.length_hi}]", "n_chunks": nmax,
                        "kept_density": pairs / (w.B * w.Hq * w.L * (w.L + 1) / 2),
                        "parallelism": f"replicas x{world} (independent layers, no collective)",
                        "l2": "inputs larger than L2 (Q+K+V = %.2f GB)" % (attn_bytes(w) / 2 / 1e9)},
