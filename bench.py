@@ -318,7 +318,7 @@ def main():
     stream = torch.cuda.current_stream()
 
     ev = lambda: torch.cuda.Event(enable_timing=True)
-    n_launch_per_step = 9   # pool x2, key norms + score tiles + select, CSR scan + fill, work list + attention
+    n_launch_per_step = 8   # pool (Q and K), key norms + score tiles + select, CSR scan + fill, work list + attention
 
     def step(timed_stages=None):
         if timed_stages is None:

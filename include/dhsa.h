@@ -96,6 +96,13 @@ int dhsa_validate_offsets(const int32_t* off, const int32_t* n_chunks, int B, in
 int dhsa_chunk_pool(const void* X, int B, int H, int L, int head_dim, const int32_t* off,
                     const int32_t* n_chunks, int Nmax, float* Xp, void* stream);
 
+/* 1b. Both poolings of a layer in one launch: Qp from Q [B, Hq, L, 128] and
+ *     Kp from K [B, Hkv, L, 128], each exactly as dhsa_chunk_pool computes it
+ *     (same arithmetic, bit-identical results). Hq % Hkv == 0; all four
+ *     pointers 16-byte aligned; errors as for dhsa_chunk_pool. */
+int dhsa_chunk_pool_qk(const void* Q, const void* K, int B, int Hq, int Hkv, int L, int head_dim,
+                       const int32_t* off, const int32_t* n_chunks, int Nmax, float* Qp, float* Kp, void* stream);
+
 /* ---------------------------------------------------------------------------
  * 2. Chunk similarity and causal per-query-chunk top-k.
  *    Source: gist.science technical summary, "Hierarchical Routing

@@ -46,6 +46,7 @@ _SIGNATURES = {
     "dhsa_check_device_status": (_I, [_P, _c.POINTER(_c.c_uint32)]),
     "dhsa_validate_offsets": (_I, [_P, _P, _I, _I, _I, _P]),
     "dhsa_chunk_pool": (_I, [_P, _I, _I, _I, _I, _P, _P, _I, _P, _P]),
+    "dhsa_chunk_pool_qk": (_I, [_P, _P, _I, _I, _I, _I, _I, _P, _P, _I, _P, _P, _P]),
     "dhsa_sel_stride": (_I, [_I, _I]),
     "dhsa_score_topk_workspace_size": (_SZ, [_I, _I, _I]),
     "dhsa_chunk_score_topk": (_I, [_P, _P, _I, _I, _I, _I, _P, _I, _P, _P, _P, _SZ, _P]),
@@ -140,6 +141,27 @@ def chunk_pool(X: torch.Tensor, off: torch.Tensor, n_chunks: torch.Tensor, out: 
     _check(load().dhsa_chunk_pool(_ptr(X), B, H, L, d, _ptr(off), _ptr(n_chunks), nmax, _ptr(out), _stream_ptr()),
            "dhsa_chunk_pool")
     return out
+
+
+def chunk_pool_qk(Q: torch.Tensor, K: torch.Tensor, off: torch.Tensor, n_chunks: torch.Tensor,
+                  Qp: Optional[torch.Tensor] = None, Kp: Optional[torch.Tensor] = None):
+    """Both poolings in one launch; same values as chunk_pool(Q) and chunk_pool(K)."""
+    B, Hq, L, d = Q.shape
+    Hkv = K.shape[1]
+    nmax = off.shape[1] - 1
+    _need(Q, torch.bfloat16, None, "Q")
+    _need(K, torch.bfloat16, (B, Hkv, L, d), "K")
+    _need(off, torch.int32, (B, nmax + 1), "off")
+    _need(n_chunks, torch.int32, (B,), "n_chunks")
+    if Qp is None:
+        Qp = torch.empty((B, Hq, nmax, d), dtype=torch.float32, device=Q.device)
+    if Kp is None:
+        Kp = torch.empty((B, Hkv, nmax, d), dtype=torch.float32, device=Q.device)
+    _need(Qp, torch.float32, (B, Hq, nmax, d), "Qp")
+    _need(Kp, torch.float32, (B, Hkv, nmax, d), "Kp")
+    _check(load().dhsa_chunk_pool_qk(_ptr(Q), _ptr(K), B, Hq, Hkv, L, d, _ptr(off), _ptr(n_chunks), nmax, _ptr(Qp),
+                                     _ptr(Kp), _stream_ptr()), "dhsa_chunk_pool_qk")
+    return Qp, Kp
 
 
 def sel_stride(k: int, nmax: int) -> int:
@@ -309,8 +331,7 @@ class DHSAPrefill:
         self.O = torch.empty((B, Hq, L, 128), dtype=torch.bfloat16, device=dev)
 
     def routing(self, Q, K):
-        chunk_pool(Q, self.off, self.n_chunks, out=self.Qp)
-        chunk_pool(K, self.off, self.n_chunks, out=self.Kp)
+        chunk_pool_qk(Q, K, self.off, self.n_chunks, Qp=self.Qp, Kp=self.Kp)
         if self.budget is None:
             chunk_score_topk(self.Qp, self.Kp, self.n_chunks, self.k, sel=self.sel, n_sel=self.n_sel,
                              workspace=self.ws_topk)

@@ -19,7 +19,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 OBJ = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libdhsa.so")
-SOURCES = ["abi.cu", "pool.cu", "score_topk.cu", "csr.cu", "attn_fwd.cu"]
+SOURCES = ["abi.cu", "pool.cu", "score_topk.cu", "csr.cu", "items.cu", "attn_fwd.cu"]
 HEADERS = ["common.cuh", "sm100_ptx.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

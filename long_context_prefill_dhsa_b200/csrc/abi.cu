@@ -8,6 +8,8 @@ namespace dhsa {
 
 int launch_chunk_pool(const void* X, int B, int H, int L, const int32_t* off, const int32_t* n_chunks, int Nmax,
                       float* Xp, cudaStream_t stream);
+int launch_chunk_pool_qk(const void* Q, const void* K, int B, int Hq, int Hkv, int L, const int32_t* off,
+                         const int32_t* n_chunks, int Nmax, float* Qp, float* Kp, cudaStream_t stream);
 int launch_validate_offsets(const int32_t* off, const int32_t* n_chunks, int B, int Nmax, int L,
                             unsigned int* status, cudaStream_t stream);
 int score_topk_stride(int k, int Nmax);
@@ -139,6 +141,18 @@ int dhsa_chunk_pool(const void* X, int B, int H, int L, int head_dim, const int3
   if (head_dim != kHeadDim) return DHSA_ERR_UNSUPPORTED;
   if ((st = check_device_sm100()) != DHSA_OK) return st;
   return launch_chunk_pool(X, B, H, L, off, n_chunks, Nmax, Xp, static_cast<cudaStream_t>(stream));
+}
+
+int dhsa_chunk_pool_qk(const void* Q, const void* K, int B, int Hq, int Hkv, int L, int head_dim,
+                       const int32_t* off, const int32_t* n_chunks, int Nmax, float* Qp, float* Kp, void* stream) {
+  int st = check_layout(B, Hq, L, Nmax, off, n_chunks);
+  if (st != DHSA_OK) return st;
+  if (Hkv <= 0 || Hq % Hkv != 0) return DHSA_ERR_INVALID_ARG;
+  if (!Q || !K || !Qp || !Kp || !aligned16(Q) || !aligned16(K) || !aligned16(Qp) || !aligned16(Kp))
+    return DHSA_ERR_INVALID_ARG;
+  if (head_dim != kHeadDim) return DHSA_ERR_UNSUPPORTED;
+  if ((st = check_device_sm100()) != DHSA_OK) return st;
+  return launch_chunk_pool_qk(Q, K, B, Hq, Hkv, L, off, n_chunks, Nmax, Qp, Kp, static_cast<cudaStream_t>(stream));
 }
 
 int dhsa_sel_stride(int k, int Nmax) {

@@ -61,11 +61,15 @@
 #include "sm100_ptx.cuh"
 
 namespace dhsa {
+
+int launch_build_items(const int32_t* off, const int32_t* n_chunks, int B, int Hq, int G, int Nmax, int4* items,
+                       int* n_items, cudaStream_t stream);
+
 namespace {
 
 using namespace ptx;
 
-constexpr int BM = 128;              // query rows per tile
+constexpr int BM = kQueryTileRows;   // query rows per tile
 constexpr int BN = 128;              // key slots per tile
 constexpr int NSK = 2;               // K pipeline stages
 constexpr int NSV = 2;               // V pipeline stages
@@ -683,62 +687,6 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_fwd_kernel(const __gr
   tmem_dealloc(tmem, kTmemCols);
 }
 
-// Work list: one item per (b, hq, chunk i, 128-row tile of i), ordered
-// (b, kv head, i, query head within the group, tile) so that CTAs running at
-// the same time share the K/V of one kv head in L2.
-__global__ void __launch_bounds__(1024) build_items_kernel(const int32_t* __restrict__ off,
-                                                           const int32_t* __restrict__ n_chunks, int B, int Hq,
-                                                           int G, int Nmax, int4* __restrict__ items,
-                                                           int* __restrict__ n_items) {
-  __shared__ int warp_sum[32];
-  __shared__ int carry_s;
-  const int t = threadIdx.x, lane = t & 31, w = t >> 5;
-  const int Hkv = Hq / G;
-  long long base = 0;
-  for (int b = 0; b < B; ++b) {
-    const int n = n_chunks[b];
-    const int32_t* ob = off + (long long)b * (Nmax + 1);
-    // pass 1: tiles of this batch element
-    int local = 0;
-    for (int c = t; c < n; c += 1024) local += (ob[c + 1] - ob[c] + BM - 1) / BM;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) local += __shfl_xor_sync(0xffffffffu, local, o);
-    if (lane == 0) warp_sum[w] = local;
-    __syncthreads();
-    int Tb = 0;
-    for (int q = 0; q < 32; ++q) Tb += warp_sum[q];
-    __syncthreads();
-    // pass 2: running exclusive scan of tiles per chunk, then write items
-    if (t == 0) carry_s = 0;
-    __syncthreads();
-    for (int c0 = 0; c0 < n; c0 += 1024) {
-      const int c = c0 + t;
-      const int tiles = (c < n) ? (ob[c + 1] - ob[c] + BM - 1) / BM : 0;
-      int incl = tiles;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int v = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += v;
-      }
-      if (lane == 31) warp_sum[w] = incl;
-      __syncthreads();
-      int before = carry_s;
-      for (int q = 0; q < w; ++q) before += warp_sum[q];
-      const int toff = before + incl - tiles;
-      for (int hkv = 0; hkv < Hkv; ++hkv)
-        for (int gq = 0; gq < G; ++gq)
-          for (int tt = 0; tt < tiles; ++tt) {
-            const long long idx = base + (long long)hkv * G * Tb + (long long)G * toff + (long long)gq * tiles + tt;
-            items[idx] = make_int4(b, hkv * G + gq, c, tt);
-          }
-      __syncthreads();
-      if (t == 1023) carry_s = before + incl;
-      __syncthreads();
-    }
-    base += (long long)Hq * Tb;
-  }
-  if (t == 0) *n_items = (int)base;
-}
 
 // --------------------------------------------------------------------- host
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -806,8 +754,7 @@ int launch_sparse_attn(const void* Q, const void* K, const void* V, int B, int H
 
   int* n_items = static_cast<int*>(ws);
   int4* items = reinterpret_cast<int4*>(static_cast<char*>(ws) + 256);
-  build_items_kernel<<<1, 1024, 0, stream>>>(off, n_chunks, B, Hq, Hq / Hkv, Nmax, items, n_items);
-  int st = launch_status();
+  int st = launch_build_items(off, n_chunks, B, Hq, Hq / Hkv, Nmax, items, n_items, stream);
   if (st != DHSA_OK) return st;
 
   int dev = 0, sms = 0;

@@ -9,6 +9,7 @@
 namespace dhsa {
 
 constexpr int kHeadDim = 128;
+constexpr int kQueryTileRows = 128;   // query rows per attention tile
 
 // Device address of the current device's status word (bits DHSA_DEVFLAG_*),
 // or nullptr with the CUDA error recorded. Kernels that can fail on the device

@@ -10,8 +10,9 @@
 // row (b, hq, i) lists the kept key chunks in ascending order.
 //
 // Two launches: a single-CTA exclusive scan of the per-row counts into
-// row_ptr, then one warp per row copying the row's chunk list and computing
-// its cost n_i * sum_j n_j (a work estimate for scheduling).
+// row_ptr (coalesced, four counts per thread per step), then one warp per row
+// copying the row's chunk list and computing its cost n_i * sum_j n_j (a
+// work estimate for scheduling).
 #include "common.cuh"
 
 namespace dhsa {
@@ -21,38 +22,52 @@ constexpr int kScanThreads = 1024;
 
 __global__ void __launch_bounds__(kScanThreads) scan_rows_kernel(const int32_t* __restrict__ n_sel, long long R,
                                                                  int32_t* __restrict__ row_ptr) {
+  // exclusive scan in blocks of 4 * kScanThreads rows: each thread reads four
+  // consecutive counts (coalesced across the block), scans them, and the
+  // block scans the thread totals; a running carry links the blocks
   __shared__ long long warp_tot[32];
+  __shared__ long long carry_s;
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-  const long long per = (R + kScanThreads - 1) / kScanThreads;
-  const long long s = t * per;
-  const long long e = (s + per < R) ? s + per : R;
-  long long local = 0;
-  for (long long r = s; r < e; ++r) local += n_sel[r];
-  long long incl = local;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const long long v = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += v;
-  }
-  if (lane == 31) warp_tot[warp] = incl;
+  if (t == 0) carry_s = 0;
   __syncthreads();
-  if (warp == 0) {
-    long long w = warp_tot[lane];
-    long long wi = w;
+  constexpr long long kChunk = 4LL * kScanThreads;
+  for (long long base = 0; base < R; base += kChunk) {
+    const long long r0 = base + 4LL * t;
+    int v[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) v[q] = (r0 + q < R) ? n_sel[r0 + q] : 0;
+    const long long local = (long long)v[0] + v[1] + v[2] + v[3];
+    long long incl = local;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      const long long v = __shfl_up_sync(0xffffffffu, wi, o);
-      if (lane >= o) wi += v;
+      const long long u = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += u;
     }
-    warp_tot[lane] = wi - w;  // exclusive prefix of the warp totals
+    if (lane == 31) warp_tot[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+      const long long w = warp_tot[lane];
+      long long wi = w;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const long long u = __shfl_up_sync(0xffffffffu, wi, o);
+        if (lane >= o) wi += u;
+      }
+      warp_tot[lane] = wi - w;  // exclusive prefix of the warp totals
+    }
+    __syncthreads();
+    const long long carry = carry_s;
+    long long run = carry + warp_tot[warp] + incl - local;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      if (r0 + q < R) row_ptr[r0 + q] = (int32_t)run;
+      run += v[q];
+    }
+    __syncthreads();                                   // everyone has read carry_s
+    if (t == kScanThreads - 1) carry_s = run;          // the last thread ends at the block total
+    __syncthreads();
   }
-  __syncthreads();
-  long long run = warp_tot[warp] + incl - local;
-  for (long long r = s; r < e; ++r) {
-    row_ptr[r] = (int32_t)run;
-    run += n_sel[r];
-  }
-  if (t == kScanThreads - 1) row_ptr[R] = (int32_t)run;
+  if (t == 0) row_ptr[R] = (int32_t)carry_s;
 }
 
 __global__ void __launch_bounds__(256) fill_rows_kernel(const int32_t* __restrict__ sel,

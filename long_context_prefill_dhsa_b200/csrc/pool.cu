@@ -26,13 +26,11 @@ __device__ __forceinline__ void add_bf16x8(float (&acc)[8], const uint4& v) {
   }
 }
 
-__global__ void __launch_bounds__(256) chunk_pool_kernel(const uint4* __restrict__ X, int H, int L,
-                                                         const int32_t* __restrict__ off,
-                                                         const int32_t* __restrict__ n_chunks, int Nmax,
-                                                         long long n_rows, float* __restrict__ Xp) {
-  const long long warp = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+// one warp pools row `warp` (= (b*H + h)*Nmax + c) of X into Xp
+__device__ __forceinline__ void pool_row(const uint4* __restrict__ X, int H, int L, const int32_t* __restrict__ off,
+                                         const int32_t* __restrict__ n_chunks, int Nmax, long long warp,
+                                         float* __restrict__ Xp) {
   const int lane = threadIdx.x & 31;
-  if (warp >= n_rows) return;
   const int c = (int)(warp % Nmax);
   const long long bh = warp / Nmax;
   const int b = (int)(bh / H);
@@ -70,6 +68,26 @@ __global__ void __launch_bounds__(256) chunk_pool_kernel(const uint4* __restrict
   }
 }
 
+__global__ void __launch_bounds__(256) chunk_pool_kernel(const uint4* __restrict__ X, int H, int L,
+                                                         const int32_t* __restrict__ off,
+                                                         const int32_t* __restrict__ n_chunks, int Nmax,
+                                                         long long n_rows, float* __restrict__ Xp) {
+  const long long warp = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  if (warp < n_rows) pool_row(X, H, L, off, n_chunks, Nmax, warp, Xp);
+}
+
+// Q and K in one launch: warps [0, rows_q) pool Q, the rest pool K, so the
+// two streams share one grid (no second launch, no tail of a small K grid).
+__global__ void __launch_bounds__(256) chunk_pool_qk_kernel(const uint4* __restrict__ Q, const uint4* __restrict__ K,
+                                                            int Hq, int Hkv, int L, const int32_t* __restrict__ off,
+                                                            const int32_t* __restrict__ n_chunks, int Nmax,
+                                                            long long rows_q, long long rows_k,
+                                                            float* __restrict__ Qp, float* __restrict__ Kp) {
+  const long long warp = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  if (warp < rows_q) pool_row(Q, Hq, L, off, n_chunks, Nmax, warp, Qp);
+  else if (warp < rows_q + rows_k) pool_row(K, Hkv, L, off, n_chunks, Nmax, warp - rows_q, Kp);
+}
+
 __global__ void validate_offsets_kernel(const int32_t* __restrict__ off, const int32_t* __restrict__ n_chunks,
                                         int B, int Nmax, int L, unsigned int* status) {
   const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
@@ -97,6 +115,17 @@ int launch_chunk_pool(const void* X, int B, int H, int L, const int32_t* off, co
   const long long blocks = (n_rows * 32 + threads - 1) / threads;
   chunk_pool_kernel<<<(unsigned)blocks, threads, 0, stream>>>(static_cast<const uint4*>(X), H, L, off, n_chunks,
                                                                Nmax, n_rows, Xp);
+  return launch_status();
+}
+
+int launch_chunk_pool_qk(const void* Q, const void* K, int B, int Hq, int Hkv, int L, const int32_t* off,
+                         const int32_t* n_chunks, int Nmax, float* Qp, float* Kp, cudaStream_t stream) {
+  const long long rows_q = (long long)B * Hq * Nmax, rows_k = (long long)B * Hkv * Nmax;
+  const int threads = 256;
+  const long long blocks = ((rows_q + rows_k) * 32 + threads - 1) / threads;
+  chunk_pool_qk_kernel<<<(unsigned)blocks, threads, 0, stream>>>(static_cast<const uint4*>(Q),
+                                                                  static_cast<const uint4*>(K), Hq, Hkv, L, off,
+                                                                  n_chunks, Nmax, rows_q, rows_k, Qp, Kp);
   return launch_status();
 }
 

@@ -273,3 +273,16 @@ def test_validate_offsets_flags_bad_table(lib):
     good = torch.tensor([[0, 5, 7, 9]], dtype=torch.int32, device="cuda")
     lib.validate_offsets(good, nc, 9)
     assert lib.check_device_status() == 0
+
+
+@needs_gpu
+def test_pool_qk_matches_separate_pools(lib):
+    """The one-launch pooling of Q and K is bit-identical to two dhsa_chunk_pool calls."""
+    w = I.custom(B=2, Hq=8, Hkv=2, L=3000, lo=1, hi=400, kind="geometric", mean=50.0, k=4, wid=112)
+    d = I.make_inputs(w)
+    t = P.to_dev(d)
+    Qp, Kp = lib.chunk_pool_qk(t["Q"], t["K"], t["off"], t["n_chunks"])
+    Qs = lib.chunk_pool(t["Q"], t["off"], t["n_chunks"])
+    Ks = lib.chunk_pool(t["K"], t["off"], t["n_chunks"])
+    torch.cuda.synchronize()
+    assert torch.equal(Qp, Qs) and torch.equal(Kp, Ks)
