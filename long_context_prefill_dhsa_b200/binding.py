@@ -348,3 +348,60 @@ class DHSAPrefill:
     def run(self, Q, K, V):
         self.routing(Q, K)
         return self.attention(Q, K, V)
+
+
+class HostStreamedPrefill:
+    """Layers whose Q, K, V arrive in pinned host memory and whose O goes back
+    to host memory, one call per layer, with the copies overlapped.
+
+    submit(Qh, Kh, Vh, Oh) enqueues: the host-to-device copy of the layer's
+    inputs on a copy-in stream, routing + attention on a compute stream, and
+    the device-to-host copy of O on a copy-out stream, chained by events.
+    Inputs and outputs are double-buffered on the device, so the copy-in of
+    layer s+1 and the copy-out of layer s-1 run while layer s computes (the
+    two copy directions use the two PCIe directions). Returns at once;
+    synchronize() waits for every submitted layer. Host buffers must stay
+    untouched until then.
+    """
+
+    def __init__(self, layer: DHSAPrefill):
+        self.layer = layer
+        dev = layer.O.device
+        B, Hq, Hkv, L = layer.B, layer.Hq, layer.Hkv, layer.L
+        self.Qd = [torch.empty((B, Hq, L, 128), dtype=torch.bfloat16, device=dev) for _ in range(2)]
+        self.Kd = [torch.empty((B, Hkv, L, 128), dtype=torch.bfloat16, device=dev) for _ in range(2)]
+        self.Vd = [torch.empty((B, Hkv, L, 128), dtype=torch.bfloat16, device=dev) for _ in range(2)]
+        self.Od = [layer.O, torch.empty_like(layer.O)]
+        self.s_in, self.s_comp, self.s_out = (torch.cuda.Stream(dev) for _ in range(3))
+        self.e_in = [torch.cuda.Event() for _ in range(2)]
+        self.e_comp = [torch.cuda.Event() for _ in range(2)]
+        self.e_out = [torch.cuda.Event() for _ in range(2)]
+        self.n = 0
+
+    def submit(self, Qh: torch.Tensor, Kh: torch.Tensor, Vh: torch.Tensor, Oh: torch.Tensor):
+        b = self.n & 1
+        lay = self.layer
+        if self.n >= 2:
+            self.s_in.wait_event(self.e_comp[b])       # layer n-2 has read this input set
+        with torch.cuda.stream(self.s_in):
+            self.Qd[b].copy_(Qh, non_blocking=True)
+            self.Kd[b].copy_(Kh, non_blocking=True)
+            self.Vd[b].copy_(Vh, non_blocking=True)
+            self.e_in[b].record(self.s_in)
+        self.s_comp.wait_event(self.e_in[b])
+        if self.n >= 2:
+            self.s_comp.wait_event(self.e_out[b])      # layer n-2's O has left this buffer
+        with torch.cuda.stream(self.s_comp):
+            lay.routing(self.Qd[b], self.Kd[b])
+            sparse_attn_fwd(self.Qd[b], self.Kd[b], self.Vd[b], lay.off, lay.n_chunks, lay.row_ptr, lay.col_idx,
+                            lay.cost, lay.scale, out=self.Od[b], workspace=lay.ws_attn)
+            self.e_comp[b].record(self.s_comp)
+        self.s_out.wait_event(self.e_comp[b])
+        with torch.cuda.stream(self.s_out):
+            Oh.copy_(self.Od[b], non_blocking=True)
+            self.e_out[b].record(self.s_out)
+        self.n += 1
+
+    def synchronize(self):
+        for s in (self.s_in, self.s_comp, self.s_out):
+            s.synchronize()

@@ -286,3 +286,31 @@ def test_pool_qk_matches_separate_pools(lib):
     Ks = lib.chunk_pool(t["K"], t["off"], t["n_chunks"])
     torch.cuda.synchronize()
     assert torch.equal(Qp, Qs) and torch.equal(Kp, Ks)
+
+
+@needs_gpu
+def test_host_streamed_layers_match_direct_runs(lib):
+    """Three layers submitted back to back from pinned host memory (copies of
+    neighbouring layers overlapping the compute) give exactly the outputs of
+    direct runs on device-resident inputs."""
+    w = I.custom(B=1, Hq=8, Hkv=2, L=4000, lo=10, hi=300, k=4, wid=113)
+    d = I.make_inputs(w)
+    t = P.to_dev(d)
+    layer = lib.DHSAPrefill(w.B, w.Hq, w.Hkv, w.L, t["off"], t["n_chunks"], w.k)
+    rng = np.random.default_rng(21)
+    hosts, refs = [], []
+    for s in range(3):
+        perm = rng.permutation(w.L)
+        hq = {x: torch.from_numpy(np.ascontiguousarray(d[x][:, :, perm])).view(torch.bfloat16).pin_memory()
+              for x in "QKV"}
+        hosts.append(hq)
+        refs.append(layer.run(*(hq[x].cuda() for x in "QKV")).clone())
+    torch.cuda.synchronize()
+    runner = lib.HostStreamedPrefill(layer)
+    outs = [torch.empty(hosts[0]["Q"].shape, dtype=torch.bfloat16).pin_memory() for _ in range(3)]
+    for hq, oh in zip(hosts, outs):
+        runner.submit(hq["Q"], hq["K"], hq["V"], oh)
+    runner.synchronize()
+    assert lib.check_device_status() == 0
+    for oh, ref in zip(outs, refs):
+        assert torch.equal(oh, ref.cpu())
