@@ -314,3 +314,26 @@ def test_host_streamed_layers_match_direct_runs(lib):
     assert lib.check_device_status() == 0
     for oh, ref in zip(outs, refs):
         assert torch.equal(oh, ref.cpu())
+
+
+@needs_gpu
+def test_graphed_layer_matches_eager(lib):
+    """A layer captured as a CUDA graph and replayed over refilled inputs gives
+    exactly the eager outputs."""
+    w = I.custom(B=2, Hq=8, Hkv=2, L=2500, lo=5, hi=200, kind="geometric", mean=60.0, k=5, wid=114)
+    d = I.make_inputs(w)
+    t = P.to_dev(d)
+    layer = lib.DHSAPrefill(w.B, w.Hq, w.Hkv, w.L, t["off"], t["n_chunks"], w.k)
+    Q, K, V = (t[x].clone() for x in "QKV")
+    g = lib.GraphedPrefill(layer, Q, K, V)
+    rng = np.random.default_rng(4)
+    for s in range(3):
+        perm = torch.from_numpy(rng.permutation(w.L)).cuda()
+        newQ, newK, newV = (t[x][:, :, perm].contiguous() for x in "QKV")
+        Q.copy_(newQ), K.copy_(newK), V.copy_(newV)
+        out = g.replay().clone()
+        ref_layer = lib.DHSAPrefill(w.B, w.Hq, w.Hkv, w.L, t["off"], t["n_chunks"], w.k)
+        ref = ref_layer.run(newQ, newK, newV)
+        torch.cuda.synchronize()
+        assert lib.check_device_status() == 0
+        assert torch.equal(out, ref)
