@@ -10,8 +10,9 @@
 // sm_100a design
 // --------------
 // * Work item = (b, hq, query chunk i, 128-row query tile of that chunk).
-//   A persistent grid (one CTA per SM) walks a work list in a static
-//   round-robin; all roles of a CTA walk the same list.
+//   A persistent grid (one CTA per SM) takes items from a work list
+//   dynamically (an atomic counter, read by each CTA's scheduler warp); the
+//   other roles follow the scheduler's ring.
 // * Key stream: the kept chunks of row (b, hq, i) are concatenated and packed
 //   into 128-slot key tiles. Each chunk starts on an 8-slot boundary (one
 //   128-byte-swizzle atom = 8 rows x 128 B, so every TMA destination is
@@ -63,7 +64,7 @@
 namespace dhsa {
 
 int launch_build_items(const int32_t* off, const int32_t* n_chunks, int B, int Hq, int G, int Nmax, int4* items,
-                       int* n_items, cudaStream_t stream);
+                       int* n_items, int* work_counter, cudaStream_t stream);
 
 namespace {
 
@@ -97,6 +98,7 @@ struct AttnParams {
   const int32_t* col_idx;
   const int4* items;      // (b, hq, i, tile)
   const int* n_items;
+  int* work_counter;      // next unassigned item (zeroed by the work-list builder)
   __nv_bfloat16* O;
   int Hq, Hkv, G, L, Nmax;
   float scale_log2;
@@ -276,10 +278,22 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_fwd_kernel(const __gr
 
   if (warp == W_SCHED) {
     // ============================================================ scheduler
+    // items are handed out dynamically: the next free item of the list goes
+    // to whichever CTA's scheduler asks first; T = -1 marks the end
     int n_local = 0;
-    for (int it = blockIdx.x; it < n_items; it += gridDim.x, ++n_local) {
+    for (;; ++n_local) {
       const int sl = n_local % NSLOT;
       if (n_local >= NSLOT && !fl.wait(bar(B_SLEMPTY + sl), ((n_local / NSLOT) - 1) & 1)) break;
+      int it = 0;
+      if (lane == 0) it = atomicAdd(p.work_counter, 1);
+      it = __shfl_sync(0xffffffffu, it, 0);
+      if (it >= n_items) {
+        if (lane == 0) {
+          slots[sl].m.T = -1;
+          mbar_arrive(bar(B_SLFULL + sl));
+        }
+        break;
+      }
       const int4 wi = p.items[it];
       const int b = wi.x, hq = wi.y, i = wi.z, tq = wi.w;
       const int32_t* ob = p.off + (long long)b * (p.Nmax + 1);
@@ -323,10 +337,11 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_fwd_kernel(const __gr
     const bool kprod = warp == W_PRODUCER;
     uint32_t g = 0;  // global key-tile counter of this CTA
     int n_local = 0;
-    for (int it = blockIdx.x; it < n_items; it += gridDim.x, ++n_local) {
+    for (;; ++n_local) {
       const int sl = n_local % NSLOT;
       if (!fl.wait(bar(B_SLFULL + sl), (n_local / NSLOT) & 1)) break;
       const ItemMeta M = slots[sl].m;
+      if (M.T < 0) break;                  // end of the work list
       const int2* seg_s = slots[sl].seg;
       const int ms = n_local & 1;
       if (kprod) {
@@ -455,10 +470,11 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_fwd_kernel(const __gr
       const uint64_t ones_desc = smem_desc_noswz(sbase + OFF_ONES, 128, 256);
       uint32_t g = 0;
       int n_local = 0;
-      for (int it = blockIdx.x; it < n_items; it += gridDim.x, ++n_local) {
+      for (;; ++n_local) {
         const int sl = n_local % NSLOT;
         if (!fl.wait(bar(B_SLFULL + sl), (n_local / NSLOT) & 1)) break;
         const int T = slots[sl].m.T;
+        if (T < 0) break;                  // end of the work list
         mbar_arrive(bar(B_SLEMPTY + sl));
         const int ms = n_local & 1;
         if (!fl.wait(bar(B_QFULL + ms), (n_local >> 1) & 1)) break;
@@ -498,10 +514,11 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_fwd_kernel(const __gr
       const uint32_t tS0 = tmem, tO = tmem + 384;
       uint32_t g = 0;
       int n_local = 0;
-      for (int it = blockIdx.x; it < n_items; it += gridDim.x, ++n_local) {
+      for (;; ++n_local) {
         const int sl = n_local % NSLOT;
         if (!fl.wait(bar(B_SLFULL + sl), (n_local / NSLOT) & 1)) break;
         const int T = slots[sl].m.T;
+        if (T < 0) break;                  // end of the work list
         mbar_arrive(bar(B_SLEMPTY + sl));
         bool ok = true;
         for (int kt = 0; kt < T; ++kt, ++g) {
@@ -544,10 +561,11 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_fwd_kernel(const __gr
     const float c = p.scale_log2;
     uint32_t g = 0;
     int n_local = 0;
-    for (int it = blockIdx.x; it < n_items; it += gridDim.x, ++n_local) {
+    for (;; ++n_local) {
       const int sl = n_local % NSLOT;
       if (!fl.wait(bar(B_SLFULL + sl), (n_local / NSLOT) & 1)) break;
       const ItemMeta M = slots[sl].m;
+      if (M.T < 0) break;                  // end of the work list
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(B_SLEMPTY + sl));
       const int qt = M.q0 + row;
@@ -753,8 +771,9 @@ int launch_sparse_attn(const void* Q, const void* K, const void* V, int B, int H
   if (!ok) return DHSA_ERR_INVALID_ARG;
 
   int* n_items = static_cast<int*>(ws);
+  int* work_counter = n_items + 1;
   int4* items = reinterpret_cast<int4*>(static_cast<char*>(ws) + 256);
-  int st = launch_build_items(off, n_chunks, B, Hq, Hq / Hkv, Nmax, items, n_items, stream);
+  int st = launch_build_items(off, n_chunks, B, Hq, Hq / Hkv, Nmax, items, n_items, work_counter, stream);
   if (st != DHSA_OK) return st;
 
   int dev = 0, sms = 0;
@@ -770,6 +789,7 @@ int launch_sparse_attn(const void* Q, const void* K, const void* V, int B, int H
   prm.col_idx = col_idx;
   prm.items = items;
   prm.n_items = n_items;
+  prm.work_counter = work_counter;
   prm.O = static_cast<__nv_bfloat16*>(O);
   prm.Hq = Hq;
   prm.Hkv = Hkv;

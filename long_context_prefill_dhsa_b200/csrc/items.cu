@@ -13,7 +13,7 @@ namespace {
 __global__ void __launch_bounds__(1024) build_items_kernel(const int32_t* __restrict__ off,
                                                            const int32_t* __restrict__ n_chunks, int B, int Hq,
                                                            int G, int Nmax, int4* __restrict__ items,
-                                                           int* __restrict__ n_items) {
+                                                           int* __restrict__ n_items, int* __restrict__ work_counter) {
   // one CTA per (query head, batch element) writes that head's items; each
   // CTA recomputes the per-chunk tile prefix of its batch element (and the
   // tile totals of the earlier ones for its base offset)
@@ -68,13 +68,15 @@ __global__ void __launch_bounds__(1024) build_items_kernel(const int32_t* __rest
     __syncthreads();
   }
   if (hq == 0 && b == B - 1 && t == 0) *n_items = (int)(base + (long long)Hq * Tb);
+  if (hq == 0 && b == 0 && t == 0) *work_counter = 0;   // the attention kernel's item dispenser
 }
 
 }  // namespace
 
 int launch_build_items(const int32_t* off, const int32_t* n_chunks, int B, int Hq, int G, int Nmax, int4* items,
-                       int* n_items, cudaStream_t stream) {
-  build_items_kernel<<<dim3(Hq, B), 1024, 0, stream>>>(off, n_chunks, B, Hq, G, Nmax, items, n_items);
+                       int* n_items, int* work_counter, cudaStream_t stream) {
+  build_items_kernel<<<dim3(Hq, B), 1024, 0, stream>>>(off, n_chunks, B, Hq, G, Nmax, items, n_items,
+                                                       work_counter);
   return launch_status();
 }
 
