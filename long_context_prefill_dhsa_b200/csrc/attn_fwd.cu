@@ -185,6 +185,25 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// maximum of 64 scores: 8 independent chains of three-input max
+__device__ __forceinline__ float max64(const uint32_t (&s)[64]) {
+  float m[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    m[e] = max3(__uint_as_float(s[e]), __uint_as_float(s[e + 8]), __uint_as_float(s[e + 16]));
+    m[e] = max3(m[e], __uint_as_float(s[e + 24]), __uint_as_float(s[e + 32]));
+    m[e] = max3(m[e], __uint_as_float(s[e + 40]), __uint_as_float(s[e + 48]));
+    m[e] = fmaxf(m[e], __uint_as_float(s[e + 56]));
+  }
+  return max3(max3(m[0], m[1], m[2]), max3(m[3], m[4], m[5]), fmaxf(m[6], m[7]));
+}
+
 // byte offset of element (row, k) in a 128 x 16 bf16 K-major block without swizzle
 __device__ __forceinline__ uint32_t noswz_off(int row, int k) {
   return (uint32_t)((row >> 3) * 256 + (k >> 3) * 128 + (row & 7) * 16 + (k & 7) * 2);
@@ -591,14 +610,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_fwd_kernel(const __gr
           for (int e = 0; e < 64; ++e)
             if (e >= thr) s[e] = __float_as_uint(-INFINITY);
         }
-        // row max over this half, 8 independent chains
-        float mx8[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) mx8[e] = __uint_as_float(s[e]);
-#pragma unroll
-        for (int cc = 8; cc < 64; ++cc) mx8[cc & 7] = fmaxf(mx8[cc & 7], __uint_as_float(s[cc]));
-        float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                         fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+        float mx = max64(s);
         // exchange the half-row maxima with the partner warp (same rows)
         xmax[(xb * 2 + half) * BM + row] = mx;
         tc_fence_before();
