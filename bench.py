@@ -34,8 +34,8 @@ ATTN_SRC = os.path.join(ROOT, "long_context_prefill_dhsa_b200", "csrc", "attn_fw
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one attention
 # launch from an ncu capture of the 32K layer, scaled by tokens (x4) to the
 # 128K layer; only valid for the kernel source it was measured on.
-ATTN_TRAFFIC = {"sha256_prefix": "b3ab6e4f140464d0",
-                "bytes_per_launch": {"llama3.1-8b-32k": 6.423e8, "llama3.1-8b-128k": 2.569e9},
+ATTN_TRAFFIC = {"sha256_prefix": "5af7e4ae8a0ac88b",
+                "bytes_per_launch": {"llama3.1-8b-32k": 6.449e8, "llama3.1-8b-128k": 2.580e9},
                 "source": "ncu --set full capture of the 32K layer; 128K scaled x4 by tokens"}
 PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS = 6650.0, 1590.0
