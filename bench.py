@@ -249,8 +249,11 @@ def cpu_oracle_sample(d, w, seconds, rule=None):
             break
     heads = w.B * w.Hq
     kv_frac = w.Hkv / w.Hq
-    est = (t_pool * (1 + kv_frac) / 2 * heads + t_route * heads + t_attn * (n / done) * heads)
+    est_route = t_pool * (1 + kv_frac) / 2 * heads + t_route * heads
+    est_attn = t_attn * (n / done) * heads
+    est = est_route + est_attn
     return {"value": est * 1e3, "unit": "ms", "cores": cores, "kind": "oracle",
+            "routing_ms": est_route * 1e3, "attention_ms": est_attn * 1e3,
             "sample": (f"oracle on (b=0, hq=0): pooling of Q and K, all {n} score/selection rows, attention of "
                        f"{done}/{n} query chunks; extrapolated x{heads} heads"
                        f"{' x' + str(round(n / done, 2)) + ' chunks' if done < n else ''}")}
