@@ -1,0 +1,157 @@
+"""The oracle's pins catch plausible mistakes.
+
+Each case swaps one function of the oracle (on the CPU, for the duration of
+the case) for a version with a typical slip -- a wrong normalisation, a
+dropped or extra term, a flipped tie rule, a shifted mask, a wrong head map
+-- and checks that at least one of the pins in test_oracle_pins.py then
+fails. Nothing here touches the CUDA library.
+"""
+import math
+
+import numpy as np
+import pytest
+
+from oracle import dhsa
+from tests import test_oracle_pins as pins
+
+_PINS = [
+    (pins.test_pool_hand_cases, {}),
+    (pins.test_pool_concat_two_equal_chunks, {}),
+    (pins.test_pool_padded_rows_zero_and_multi_batch, {}),
+    (pins.test_select_matches_bruteforce_block_mask, {"c": 4, "m": 12, "k": 3, "G": 1}),
+    (pins.test_select_matches_bruteforce_block_mask, {"c": 5, "m": 16, "k": 5, "G": 4}),
+    (pins.test_select_ties_go_to_lower_index, {}),
+    (pins.test_select_edges, {}),
+    (pins.test_csr_by_hand, {}),
+    (pins.test_kept_pairs_by_hand, {}),
+    (pins.test_attn_k_all_equals_dense, {}),
+    (pins.test_attn_k0_is_per_chunk_causal, {}),
+    (pins.test_attn_matches_explicit_token_mask, {}),
+    (pins.test_attn_single_token_and_convexity, {}),
+    (pins.test_budget_hand_cases, {}),
+    (pins.test_budget_reduces_to_topk, {"seed": 0}),
+    (pins.test_budget_uniform_lengths_is_topk_of_budget_over_length, {}),
+    (pins.test_budget_zero_keeps_recent_window_only, {}),
+    (pins.test_budget_invariants_random, {}),
+]
+
+
+def _failing_pins():
+    failed = []
+    for fn, kw in _PINS:
+        try:
+            fn(**kw)
+        except Exception:          # an assertion or an error the slip provokes
+            failed.append(fn.__name__)
+    return failed
+
+
+# ------------------------------------------------------------ the slips
+def _pool_mean(X, off, n_chunks, nmax):
+    """Mean instead of mean * sqrt(n)."""
+    P = _orig["chunk_pool"](X, off, n_chunks, nmax)
+    out = P.copy()
+    for b in range(off.shape[0]):
+        for c in range(int(n_chunks[b])):
+            out[b, :, c] = P[b, :, c] / math.sqrt(int(off[b, c + 1] - off[b, c]))
+    return out
+
+
+def _pool_sum(X, off, n_chunks, nmax):
+    """Plain sum: the 1/sqrt(n) dropped."""
+    P = _orig["chunk_pool"](X, off, n_chunks, nmax)
+    out = P.copy()
+    for b in range(off.shape[0]):
+        for c in range(int(n_chunks[b])):
+            out[b, :, c] = P[b, :, c] * math.sqrt(int(off[b, c + 1] - off[b, c]))
+    return out
+
+
+def _scores_wrong_group(Qp, Kp, n_chunks):
+    """Query head hq scored against kv head hq % Hkv instead of hq // G."""
+    B, Hq, nmax, _ = Qp.shape
+    Hkv = Kp.shape[1]
+    Kr = Kp[:, [h % Hkv for h in range(Hq)]]
+    S = np.zeros((B, Hq, nmax, nmax))
+    for b in range(B):
+        S[b] = np.einsum("hid,hjd->hij", Qp[b], Kr[b])
+    mask = np.tril(np.ones((nmax, nmax), dtype=bool), k=-1)
+    return np.where(mask[None, None], S, 0.0)
+
+
+def _select_ties_high(S_row, i, k):
+    """Ties to the higher chunk index."""
+    cand = np.arange(i)[::-1]
+    order = cand[np.argsort(-S_row[:i][::-1], kind="stable")]
+    keep = np.sort(order[: min(k, i)])
+    return np.concatenate([keep, [i]]).astype(np.int64)
+
+
+def _select_one_more(S_row, i, k):
+    """k + 1 earlier chunks."""
+    return _orig["select_row"](S_row, i, k + 1)
+
+
+def _select_no_diag(S_row, i, k):
+    """The diagonal chunk left out when there are earlier chunks."""
+    r = _orig["select_row"](S_row, i, k)
+    return r[:-1] if len(r) > 1 else r
+
+
+def _attn_scale_sq(Q, K, V, off_b, kept, i, scale, dtype=np.float64):
+    """Scores scaled by 1/d instead of 1/sqrt(d)."""
+    return _orig["attn_chunk"](Q, K, V, off_b, kept, i, scale * scale, dtype)
+
+
+def _attn_strict_causal(Q, K, V, off_b, kept, i, scale, dtype=np.float64):
+    """Key s visible to query t only if s < t (a token no longer sees itself)."""
+    qs, qe = dhsa.chunk_bounds(off_b, i)
+    rows = np.concatenate([np.arange(*dhsa.chunk_bounds(off_b, int(j))) for j in kept])
+    q, k, v = Q[qs:qe].astype(dtype), K[rows].astype(dtype), V[rows].astype(dtype)
+    logits = (q @ k.T) * dtype(scale)
+    t = np.arange(qs, qe)[:, None]
+    logits = np.where(rows[None, :] < t, logits, -np.inf)
+    m = np.max(np.where(np.isfinite(logits), logits, -1e300), axis=1, keepdims=True)
+    p = np.where(np.isfinite(logits), np.exp(logits - m), 0.0)
+    den = p.sum(axis=1, keepdims=True)
+    return (p @ v) / np.where(den > 0, den, 1.0)
+
+
+def _budget_strict(S_row, lens, i, budget, recent, k_max):
+    """Stops only once the kept tokens exceed the budget (> instead of >=)."""
+    return _orig["select_budget_row"](S_row, lens, i, budget + 1, recent, k_max)
+
+
+def _budget_window_uncounted(S_row, lens, i, budget, recent, k_max):
+    """The recent window's tokens not counted against the budget."""
+    r = min(recent, i, k_max)
+    extra = int(sum(int(lens[j]) for j in range(i - r, i)))
+    return _orig["select_budget_row"](S_row, lens, i, budget + extra, recent, k_max)
+
+
+_orig = {name: getattr(dhsa, name) for name in
+         ("chunk_pool", "chunk_scores", "select_row", "attn_chunk", "select_budget_row")}
+
+SLIPS = [
+    ("chunk_pool", _pool_mean),
+    ("chunk_pool", _pool_sum),
+    ("chunk_scores", _scores_wrong_group),
+    ("select_row", _select_ties_high),
+    ("select_row", _select_one_more),
+    ("select_row", _select_no_diag),
+    ("attn_chunk", _attn_scale_sq),
+    ("attn_chunk", _attn_strict_causal),
+    ("select_budget_row", _budget_strict),
+    ("select_budget_row", _budget_window_uncounted),
+]
+
+
+def test_pins_pass_on_the_oracle_as_written():
+    assert _failing_pins() == []
+
+
+@pytest.mark.parametrize("name,slip", SLIPS, ids=[s[1].__name__ for s in SLIPS])
+def test_a_slip_fails_some_pin(monkeypatch, name, slip):
+    monkeypatch.setattr(dhsa, name, slip)
+    failed = _failing_pins()
+    assert failed, f"no pin caught {slip.__name__}: {slip.__doc__}"
