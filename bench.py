@@ -33,8 +33,9 @@ METRIC = "ms per layer (mask+attn) and TFLOP/s on kept pairs at 128K, % of roofl
 ATTN_SRC = os.path.join(ROOT, "long_context_prefill_dhsa_b200", "csrc", "attn_fwd.cu")
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one attention
 # launch from an ncu capture of the 32K layer, scaled by tokens (x4) to the
-# 128K layer; only valid for the kernel source it was measured on.
-ATTN_TRAFFIC = {"sha256_prefix": "5af7e4ae8a0ac88b",
+# 128K layer; only valid for the kernel source it was measured on (the sha256
+# of the kernel's constants and body, see kernel_region_sha).
+ATTN_TRAFFIC = {"sha256_prefix": "477f3c53f602489b",
                 "bytes_per_launch": {"llama3.1-8b-32k": 6.449e8, "llama3.1-8b-128k": 2.580e9},
                 "source": "ncu --set full capture of the 32K layer; 128K scaled x4 by tokens"}
 PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -59,6 +60,9 @@ def parse():
     ap.add_argument("--recent", type=int, default=0)
     ap.add_argument("--kmax", type=int, default=None)
     ap.add_argument("--budget-spread", type=float, default=0.0)
+    # query-tile policy of the attention: 0 = 128-row tiles (default, fastest);
+    # 1 = chunk tails of at most 64 rows on the 64-row kernel; 2 = 64-row tiles only
+    ap.add_argument("--short-tiles", type=int, default=0, choices=[0, 1, 2])
     return ap.parse_args()
 
 
@@ -77,9 +81,19 @@ def selection_rule(args, w, nmax):
     return k_max, args.budget, args.recent, desc
 
 
-def attn_traffic(workload_name):
+def kernel_region_sha(path=ATTN_SRC):
+    """sha256 prefix of the attention kernel's device code: from its
+    constants (`using namespace ptx;`) through the kernel's closing brace.
+    Host-side launch code after the kernel does not enter it."""
     import hashlib
-    sha = hashlib.sha256(open(ATTN_SRC, "rb").read()).hexdigest()[:16]
+    s = open(path).read()
+    a = s.index("using namespace ptx;")
+    b = s.index("\n}\n", s.index("__global__", a)) + 3
+    return hashlib.sha256(s[a:b].encode()).hexdigest()[:16]
+
+
+def attn_traffic(workload_name):
+    sha = kernel_region_sha()
     if sha != ATTN_TRAFFIC["sha256_prefix"]:
         return None, "kernel changed since the ncu capture"
     v = ATTN_TRAFFIC["bytes_per_launch"].get(workload_name)
@@ -317,11 +331,14 @@ def main():
     off, nc = host_off.to(dev), host_nc.to(dev)
     k_sel, bud, recent, sel_desc = selection_rule(args, w, d["off"].shape[1] - 1)
     bud_arg = torch.from_numpy(bud).to(dev) if isinstance(bud, np.ndarray) else bud
-    layer = binding.DHSAPrefill(w.B, w.Hq, w.Hkv, w.L, off, nc, k_sel, device=dev, budget=bud_arg, recent=recent)
+    layer = binding.DHSAPrefill(w.B, w.Hq, w.Hkv, w.L, off, nc, k_sel, device=dev, budget=bud_arg, recent=recent,
+                                short_tiles=args.short_tiles)
     stream = torch.cuda.current_stream()
 
     ev = lambda: torch.cuda.Event(enable_timing=True)
-    n_launch_per_step = 8   # pool (Q and K), key norms + score tiles + select, CSR scan + fill, work list + attention
+    # pool (Q and K), key norms + score tiles + select, CSR scan + fill, work list + attention
+    # (tile policy 1 launches both attention kernels)
+    n_launch_per_step = 8 + (1 if args.short_tiles == 1 else 0)
 
     def step(timed_stages=None):
         if timed_stages is None:
@@ -365,6 +382,8 @@ def main():
     attn_tflops = flop / (attn_ms * 1e-3) / 1e12
     rbytes = routing_bytes(w, nmax, k_sel)
     traffic, traffic_src = attn_traffic(w.name)
+    if args.short_tiles:
+        traffic, traffic_src = None, "captured for the 128-row tile policy only"
 
     # end to end through the public API with host buffers (pinned), on this rank:
     # every step copies that layer's Q, K, V in from pinned host memory and its
@@ -436,13 +455,17 @@ def main():
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "L": w.L, "head_dim": 128,
                        "k": w.k, "selection": sel_desc,
+                       "query_tiles": ["128 rows", "128 rows, tails <= 64 rows on the 64-row kernel",
+                                       "64 rows"][args.short_tiles],
                        "chunk_len": f"{w.length_kind}[{w.length_lo},{w.length_hi}]", "n_chunks": nmax,
                        "kept_density": pairs / (w.B * w.Hq * w.L * (w.L + 1) / 2),
                        "parallelism": f"replicas x{world} (independent layers, no collective)",
                        "l2": "inputs larger than L2 (Q+K+V = %.2f GB)" % (attn_bytes(w) / 2 / 1e9)},
             "stages_ms": {"routing": route_ms, "attention": attn_ms},
             "tflops_kept_pairs": flop / (ms_step * 1e-3) / 1e12,
-            "roofline": {"bound": "tensor", "kernel": "sparse_attn_fwd_kernel", "achieved": attn_tflops,
+            "roofline": {"bound": "tensor", "achieved": attn_tflops,
+                         "kernel": ["sparse_attn_fwd_kernel", "sparse_attn_fwd_kernel + sparse_attn_short_kernel",
+                                    "sparse_attn_short_kernel"][args.short_tiles],
                          "peak": tc_peak, "unit": "TFLOP/s", "frac": attn_tflops / tc_peak,
                          "peak_kind": f"{peak_kind} bf16 dense (burst)", "traffic": traffic,
                          "traffic_source": traffic_src, "flop_per_launch": flop},

@@ -223,7 +223,7 @@ int dhsa_sparse_attn_fwd(const void* Q, const void* K, const void* V, int B, int
  *    in `workspace` is kept instead in a 4 MiB static device array of the
  *    library (held by every GPU that loads the library until process exit).
  *    Problems whose work list does not fit, i.e.
- *      256 + 16 * B * Hq * (Nmax + ceil(L / 128)) > 4 MiB,
+ *      dhsa_sparse_attn_workspace_size(B, Hq, L, Nmax) > 4 MiB,
  *    are rejected with DHSA_ERR_WORKSPACE before anything is enqueued
  *    (use 4. for those). This call performs no cudaMalloc/cudaFree and calls
  *    no allocating library routine.
@@ -242,6 +242,33 @@ int dhsa_sparse_attn_fwd_noalloc(const void* Q, const void* K, const void* V, in
                                  int head_dim, const int32_t* off, const int32_t* n_chunks, int Nmax,
                                  const int32_t* row_ptr, const int32_t* col_idx, float softmax_scale, void* O,
                                  void* stream);
+
+/* ---------------------------------------------------------------------------
+ * 4c. The same attention forward with a choice of query-tile shapes.
+ *    The paper has no counterpart: the DHSA README ("Overview") stresses that
+ *    chunks are variable-sized, and a chunk whose last 128-row query tile
+ *    holds few rows leaves most of that tile idle. This entry can hand such
+ *    rows to a second kernel whose tiles hold at most 64 query rows (keys on
+ *    the tensor core's M side, queries on its N side).
+ *
+ *    short_tiles: 0 = every query tile has 128 rows (this is
+ *    dhsa_sparse_attn_fwd); 1 = a chunk's last tile goes to the 64-row kernel
+ *    when it holds at most 64 rows; 2 = every chunk is cut into 64-row tiles.
+ *    Other values: DHSA_ERR_INVALID_ARG. The output is the same computation
+ *    for every choice (the order of the fp32 sums differs, so results may
+ *    differ in the last bf16 place). On B200 the 64-row kernel is not faster
+ *    per query row than the 128-row one (its two MMAs both stream their
+ *    operands from shared memory), so 0 is the fast choice.
+ *
+ *    workspace: dhsa_sparse_attn_tiles_workspace_size(B, Hq, L, Nmax,
+ *    short_tiles) bytes (0 for invalid arguments). Other arguments, layouts,
+ *    results and errors as for dhsa_sparse_attn_fwd.
+ * ------------------------------------------------------------------------- */
+size_t dhsa_sparse_attn_tiles_workspace_size(int B, int Hq, int L, int Nmax, int short_tiles);
+int dhsa_sparse_attn_fwd_tiles(const void* Q, const void* K, const void* V, int B, int Hq, int Hkv, int L,
+                               int head_dim, const int32_t* off, const int32_t* n_chunks, int Nmax,
+                               const int32_t* row_ptr, const int32_t* col_idx, float softmax_scale, int short_tiles,
+                               void* O, void* workspace, size_t workspace_bytes, void* stream);
 
 #ifdef __cplusplus
 }

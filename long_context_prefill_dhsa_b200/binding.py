@@ -57,6 +57,9 @@ _SIGNATURES = {
     "dhsa_sparse_attn_workspace_size": (_SZ, [_I, _I, _I, _I]),
     "dhsa_sparse_attn_fwd": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _I, _P, _P, _P, _F, _P, _P, _SZ, _P]),
     "dhsa_sparse_attn_fwd_noalloc": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _I, _P, _P, _F, _P, _P]),
+    "dhsa_sparse_attn_tiles_workspace_size": (_SZ, [_I, _I, _I, _I, _I]),
+    "dhsa_sparse_attn_fwd_tiles": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _I, _P, _P, _F, _I, _P, _P, _SZ,
+                                        _P]),
 }
 
 _lib: Optional[ctypes.CDLL] = None
@@ -252,7 +255,10 @@ def build_block_csr(sel: torch.Tensor, n_sel: torch.Tensor, k: int, off: torch.T
 def sparse_attn_fwd(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, off: torch.Tensor, n_chunks: torch.Tensor,
                     row_ptr: torch.Tensor, col_idx: torch.Tensor, cost: Optional[torch.Tensor] = None,
                     softmax_scale: Optional[float] = None, out: Optional[torch.Tensor] = None,
-                    workspace: Optional[torch.Tensor] = None):
+                    workspace: Optional[torch.Tensor] = None, short_tiles: int = 0):
+    """Attention over the kept chunk pairs. short_tiles != 0 calls the
+    tile-policy entry (include/dhsa.h, 4c): 1 sends chunk tails of at most 64
+    rows, 2 every row, to the 64-row kernel."""
     B, Hq, L, d = Q.shape
     Hkv = K.shape[1]
     nmax = off.shape[1] - 1
@@ -263,13 +269,19 @@ def sparse_attn_fwd(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, off: torc
     if out is None:
         out = torch.empty_like(Q)
     _need(out, torch.bfloat16, (B, Hq, L, d), "out")
-    ws_bytes = lib.dhsa_sparse_attn_workspace_size(B, Hq, L, nmax)
+    ws_bytes = lib.dhsa_sparse_attn_tiles_workspace_size(B, Hq, L, nmax, short_tiles)
     if workspace is None:
-        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=Q.device)
+        workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=Q.device)
     scale = 1.0 / math.sqrt(d) if softmax_scale is None else float(softmax_scale)
-    _check(lib.dhsa_sparse_attn_fwd(_ptr(Q), _ptr(K), _ptr(V), B, Hq, Hkv, L, d, _ptr(off), _ptr(n_chunks), nmax,
-                                    _ptr(row_ptr), _ptr(col_idx), _ptr(cost), scale, _ptr(out), _ptr(workspace),
-                                    workspace.numel(), _stream_ptr()), "dhsa_sparse_attn_fwd")
+    if short_tiles == 0:
+        _check(lib.dhsa_sparse_attn_fwd(_ptr(Q), _ptr(K), _ptr(V), B, Hq, Hkv, L, d, _ptr(off), _ptr(n_chunks),
+                                        nmax, _ptr(row_ptr), _ptr(col_idx), _ptr(cost), scale, _ptr(out),
+                                        _ptr(workspace), workspace.numel(), _stream_ptr()), "dhsa_sparse_attn_fwd")
+    else:
+        _check(lib.dhsa_sparse_attn_fwd_tiles(_ptr(Q), _ptr(K), _ptr(V), B, Hq, Hkv, L, d, _ptr(off),
+                                              _ptr(n_chunks), nmax, _ptr(row_ptr), _ptr(col_idx), scale,
+                                              int(short_tiles), _ptr(out), _ptr(workspace), workspace.numel(),
+                                              _stream_ptr()), "dhsa_sparse_attn_fwd_tiles")
     return out
 
 
@@ -304,12 +316,16 @@ class DHSAPrefill:
     Selection is the top-k rule, or, when `budget` is given (an int, or an
     int32 tensor [B, Hq, Nmax] of per-row budgets), the token-budget rule with
     a window of `recent` chunks and at most k earlier chunks per row.
+    `short_tiles` picks the query-tile policy of the attention (0: 128-row
+    tiles only, the fast default; 1 and 2: see sparse_attn_fwd).
     """
 
     def __init__(self, B: int, Hq: int, Hkv: int, L: int, off: torch.Tensor, n_chunks: torch.Tensor, k: int,
-                 device="cuda", softmax_scale: Optional[float] = None, budget=None, recent: int = 0):
+                 device="cuda", softmax_scale: Optional[float] = None, budget=None, recent: int = 0,
+                 short_tiles: int = 0):
         lib = load()
         self.B, self.Hq, self.Hkv, self.L, self.k = B, Hq, Hkv, L, k
+        self.short_tiles = short_tiles
         self.budget, self.recent = budget, recent
         self.off, self.n_chunks = off, n_chunks
         self.nmax = off.shape[1] - 1
@@ -326,8 +342,8 @@ class DHSAPrefill:
         self.row_ptr = torch.empty(B * Hq * nmax + 1, dtype=torch.int32, device=dev)
         self.col_idx = torch.empty(lib.dhsa_csr_nnz_upper(B, Hq, nmax, k), dtype=torch.int32, device=dev)
         self.cost = torch.empty(B * Hq * nmax, dtype=torch.int64, device=dev)
-        self.ws_attn = torch.empty(lib.dhsa_sparse_attn_workspace_size(B, Hq, L, nmax), dtype=torch.uint8,
-                                   device=dev)
+        self.ws_attn = torch.empty(max(lib.dhsa_sparse_attn_tiles_workspace_size(B, Hq, L, nmax, short_tiles), 1),
+                                   dtype=torch.uint8, device=dev)
         self.O = torch.empty((B, Hq, L, 128), dtype=torch.bfloat16, device=dev)
 
     def routing(self, Q, K):
@@ -343,7 +359,7 @@ class DHSAPrefill:
 
     def attention(self, Q, K, V):
         return sparse_attn_fwd(Q, K, V, self.off, self.n_chunks, self.row_ptr, self.col_idx, self.cost,
-                               self.scale, out=self.O, workspace=self.ws_attn)
+                               self.scale, out=self.O, workspace=self.ws_attn, short_tiles=self.short_tiles)
 
     def run(self, Q, K, V):
         self.routing(Q, K)

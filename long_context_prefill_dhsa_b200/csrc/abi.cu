@@ -23,11 +23,11 @@ int launch_score_budget(const float* Qp, const float* Kp, int B, int Hq, int Hkv
 int launch_build_csr(const int32_t* sel, const int32_t* n_sel, int B, int Hq, int Nmax, int k, const int32_t* off,
                      const int32_t* n_chunks, int32_t* row_ptr, int32_t* col_idx, int64_t* cost,
                      unsigned int* status, cudaStream_t stream);
-size_t attn_ws_bytes(int B, int Hq, int L, int Nmax);
+size_t attn_ws_bytes(int B, int Hq, int L, int Nmax, int policy);
 int launch_sparse_attn(const void* Q, const void* K, const void* V, int B, int Hq, int Hkv, int L,
                        const int32_t* off, const int32_t* n_chunks, int Nmax, const int32_t* row_ptr,
-                       const int32_t* col_idx, float softmax_scale, void* O, void* ws, unsigned int* status,
-                       cudaStream_t stream);
+                       const int32_t* col_idx, float softmax_scale, int policy, void* O, void* ws,
+                       unsigned int* status, cudaStream_t stream);
 size_t noalloc_scratch_bytes();
 int noalloc_scratch_ptr(void** out);
 
@@ -216,8 +216,12 @@ int dhsa_build_block_csr(const int32_t* sel, const int32_t* n_sel, int B, int Hq
 }
 
 size_t dhsa_sparse_attn_workspace_size(int B, int Hq, int L, int Nmax) {
-  if (B <= 0 || Hq <= 0 || L <= 0 || Nmax <= 0) return 0;
-  return attn_ws_bytes(B, Hq, L, Nmax);
+  return dhsa_sparse_attn_tiles_workspace_size(B, Hq, L, Nmax, 0);
+}
+
+size_t dhsa_sparse_attn_tiles_workspace_size(int B, int Hq, int L, int Nmax, int short_tiles) {
+  if (B <= 0 || Hq <= 0 || L <= 0 || Nmax <= 0 || short_tiles < 0 || short_tiles > 2) return 0;
+  return attn_ws_bytes(B, Hq, L, Nmax, short_tiles);
 }
 
 int dhsa_sparse_attn_fwd(const void* Q, const void* K, const void* V, int B, int Hq, int Hkv, int L, int head_dim,
@@ -225,20 +229,29 @@ int dhsa_sparse_attn_fwd(const void* Q, const void* K, const void* V, int B, int
                          const int32_t* col_idx, const int64_t* cost, float softmax_scale, void* O, void* workspace,
                          size_t workspace_bytes, void* stream) {
   (void)cost;
+  return dhsa_sparse_attn_fwd_tiles(Q, K, V, B, Hq, Hkv, L, head_dim, off, n_chunks, Nmax, row_ptr, col_idx,
+                                    softmax_scale, 0, O, workspace, workspace_bytes, stream);
+}
+
+int dhsa_sparse_attn_fwd_tiles(const void* Q, const void* K, const void* V, int B, int Hq, int Hkv, int L,
+                               int head_dim, const int32_t* off, const int32_t* n_chunks, int Nmax,
+                               const int32_t* row_ptr, const int32_t* col_idx, float softmax_scale, int short_tiles,
+                               void* O, void* workspace, size_t workspace_bytes, void* stream) {
   int st = check_layout(B, Hq, L, Nmax, off, n_chunks);
   if (st != DHSA_OK) return st;
   if (!Q || !K || !V || !O || !row_ptr || !col_idx) return DHSA_ERR_INVALID_ARG;
   if (Hkv <= 0 || Hq % Hkv != 0) return DHSA_ERR_INVALID_ARG;
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O)) return DHSA_ERR_INVALID_ARG;
   if (!(softmax_scale > 0.f) || softmax_scale != softmax_scale) return DHSA_ERR_INVALID_ARG;
+  if (short_tiles < 0 || short_tiles > 2) return DHSA_ERR_INVALID_ARG;
   if (head_dim != kHeadDim) return DHSA_ERR_UNSUPPORTED;
-  if (!workspace || workspace_bytes < attn_ws_bytes(B, Hq, L, Nmax) || !aligned16(workspace))
+  if (!workspace || workspace_bytes < attn_ws_bytes(B, Hq, L, Nmax, short_tiles) || !aligned16(workspace))
     return DHSA_ERR_WORKSPACE;
   if ((st = check_device_sm100()) != DHSA_OK) return st;
   unsigned int* status = device_status_ptr();
   if (!status) return DHSA_ERR_CUDA;
-  return launch_sparse_attn(Q, K, V, B, Hq, Hkv, L, off, n_chunks, Nmax, row_ptr, col_idx, softmax_scale, O,
-                            workspace, status, static_cast<cudaStream_t>(stream));
+  return launch_sparse_attn(Q, K, V, B, Hq, Hkv, L, off, n_chunks, Nmax, row_ptr, col_idx, softmax_scale,
+                            short_tiles, O, workspace, status, static_cast<cudaStream_t>(stream));
 }
 
 int dhsa_sparse_attn_fwd_noalloc(const void* Q, const void* K, const void* V, int B, int Hq, int Hkv, int L,
@@ -252,13 +265,13 @@ int dhsa_sparse_attn_fwd_noalloc(const void* Q, const void* K, const void* V, in
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O)) return DHSA_ERR_INVALID_ARG;
   if (!(softmax_scale > 0.f) || softmax_scale != softmax_scale) return DHSA_ERR_INVALID_ARG;
   if (head_dim != kHeadDim) return DHSA_ERR_UNSUPPORTED;
-  if (attn_ws_bytes(B, Hq, L, Nmax) > noalloc_scratch_bytes()) return DHSA_ERR_WORKSPACE;
+  if (attn_ws_bytes(B, Hq, L, Nmax, 0) > noalloc_scratch_bytes()) return DHSA_ERR_WORKSPACE;
   if ((st = check_device_sm100()) != DHSA_OK) return st;
   unsigned int* status = device_status_ptr();
   if (!status) return DHSA_ERR_CUDA;
   void* scratch = nullptr;
   if ((st = noalloc_scratch_ptr(&scratch)) != DHSA_OK) return st;
-  return launch_sparse_attn(Q, K, V, B, Hq, Hkv, L, off, n_chunks, Nmax, row_ptr, col_idx, softmax_scale, O,
+  return launch_sparse_attn(Q, K, V, B, Hq, Hkv, L, off, n_chunks, Nmax, row_ptr, col_idx, softmax_scale, 0, O,
                             scratch, status, static_cast<cudaStream_t>(stream));
 }
 

@@ -60,12 +60,9 @@
 
 #include "common.cuh"
 #include "sm100_ptx.cuh"
+#include "tmap.cuh"
 
 namespace dhsa {
-
-int launch_build_items(const int32_t* off, const int32_t* n_chunks, int B, int Hq, int G, int Nmax, int4* items,
-                       int* n_items, int* work_counter, cudaStream_t stream);
-
 namespace {
 
 using namespace ptx;
@@ -718,75 +715,24 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_fwd_kernel(const __gr
 }
 
 
-// --------------------------------------------------------------------- host
-using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn get_encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (!fn) {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(ptr);
-  }
-  return fn;
-}
-
-bool make_map(EncodeTiledFn enc, CUtensorMap* m, const void* base, long long rows, int box_rows) {
-  const cuuint64_t dims[2] = {(cuuint64_t)kHeadDim, (cuuint64_t)rows};
-  const cuuint64_t strides[1] = {(cuuint64_t)kHeadDim * 2};
-  const cuuint32_t box[2] = {64u, (cuuint32_t)box_rows};
-  const cuuint32_t estr[2] = {1u, 1u};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 }  // namespace
 
-// ----------------------------------------------------------- no-allocation variant
-// Scratch for callers that must not allocate device memory. It lives in a
-// file-scope device array that every GPU loading the library holds until the
-// process exits. It backs the same work list the caller's workspace would
-// hold, so the maximum problem is the one whose work list fits:
-// 256 + 16 * B * Hq * (Nmax + ceil(L / 128)) bytes <= 4 MiB.
-constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;
-static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
-
-namespace {
-constexpr int kNoAllocMaxDevices = 64;
-void* g_noalloc_ptr[kNoAllocMaxDevices] = {nullptr};
-}  // namespace
-
-size_t attn_items_cap(int B, int Hq, int L, int Nmax) {
-  return (size_t)B * Hq * ((size_t)Nmax + (size_t)(L + BM - 1) / BM);
-}
-
-size_t attn_ws_bytes(int B, int Hq, int L, int Nmax) { return 256 + sizeof(int4) * attn_items_cap(B, Hq, L, Nmax); }
-
-int launch_sparse_attn(const void* Q, const void* K, const void* V, int B, int Hq, int Hkv, int L,
-                       const int32_t* off, const int32_t* n_chunks, int Nmax, const int32_t* row_ptr,
-                       const int32_t* col_idx, float softmax_scale, void* O, void* ws, unsigned int* status,
-                       cudaStream_t stream) {
-  EncodeTiledFn enc = get_encode_fn();
+// Launches the persistent kernel over the long work list (built beforehand
+// on the same stream). Returns DHSA_OK or the launch error.
+int launch_sparse_attn_long(const AttnWork& w, const void* Q, const void* K, const void* V, int B, int Hq, int Hkv,
+                            int L, const int32_t* off, int Nmax, const int32_t* row_ptr, const int32_t* col_idx,
+                            float softmax_scale, void* O, unsigned int* status, cudaStream_t stream) {
+  if (w.cap_long == 0) return DHSA_OK;
+  EncodeTiledFn enc = tmap_encode_fn();
   if (!enc) return cuda_status(cudaErrorNotSupported);
   AttnMaps maps;
   const long long q_rows = (long long)B * Hq * L, kv_rows = (long long)B * Hkv * L;
-  bool ok = make_map(enc, &maps.q, Q, q_rows, BM);
+  bool ok = make_rows_map(enc, &maps.q, Q, q_rows, BM);
   for (int s = 0; s < 16; ++s) {
-    ok = ok && make_map(enc, &maps.k[s], K, kv_rows, 8 * (s + 1));
-    ok = ok && make_map(enc, &maps.v[s], V, kv_rows, 8 * (s + 1));
+    ok = ok && make_rows_map(enc, &maps.k[s], K, kv_rows, 8 * (s + 1));
+    ok = ok && make_rows_map(enc, &maps.v[s], V, kv_rows, 8 * (s + 1));
   }
   if (!ok) return DHSA_ERR_INVALID_ARG;
-
-  int* n_items = static_cast<int*>(ws);
-  int* work_counter = n_items + 1;
-  int4* items = reinterpret_cast<int4*>(static_cast<char*>(ws) + 256);
-  int st = launch_build_items(off, n_chunks, B, Hq, Hq / Hkv, Nmax, items, n_items, work_counter, stream);
-  if (st != DHSA_OK) return st;
 
   int dev = 0, sms = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -799,9 +745,9 @@ int launch_sparse_attn(const void* Q, const void* K, const void* V, int B, int H
   prm.off = off;
   prm.row_ptr = row_ptr;
   prm.col_idx = col_idx;
-  prm.items = items;
-  prm.n_items = n_items;
-  prm.work_counter = work_counter;
+  prm.items = w.items_long;
+  prm.n_items = w.n_long;
+  prm.work_counter = w.counter_long;
   prm.O = static_cast<__nv_bfloat16*>(O);
   prm.Hq = Hq;
   prm.Hkv = Hkv;
@@ -810,34 +756,9 @@ int launch_sparse_attn(const void* Q, const void* K, const void* V, int B, int H
   prm.Nmax = Nmax;
   prm.scale_log2 = softmax_scale * 1.4426950408889634f;
   prm.status = status;
-  const long long cap = (long long)attn_items_cap(B, Hq, L, Nmax);
-  const int grid = (int)(cap < sms ? cap : sms);
+  const int grid = (int)(w.cap_long < sms ? w.cap_long : sms);
   sparse_attn_fwd_kernel<<<grid, kThreads, kSmemAlloc, stream>>>(maps, prm);
   return launch_status();
-}
-
-}  // namespace dhsa
-
-namespace dhsa {
-
-size_t noalloc_scratch_bytes() { return kNoAllocScratchBytes; }
-
-// Device address of the static scratch on the current device. The host-side
-// name g_noalloc_scratch is only a stand-in, so the address is looked up once
-// per device (on that device's first call) and cached.
-int noalloc_scratch_ptr(void** out) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return cuda_status(e);
-  if (dev < 0 || dev >= kNoAllocMaxDevices) return DHSA_ERR_UNSUPPORTED;
-  if (!g_noalloc_ptr[dev]) {
-    void* ptr = nullptr;
-    e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
-    if (e != cudaSuccess) return cuda_status(e);
-    g_noalloc_ptr[dev] = ptr;
-  }
-  *out = g_noalloc_ptr[dev];
-  return DHSA_OK;
 }
 
 }  // namespace dhsa

@@ -217,3 +217,22 @@ def custom(B=1, Hq=2, Hkv=1, L=256, lo=1, hi=64, kind="uniform", mean=0.0, k=4,
     """A small workload for edge cases (ragged tails, one-row chunks, ...)."""
     return Workload(wid, name, B, Hq, Hkv, L, kind, lo, hi, length_mean=mean, k=k,
                     needles_per_head=needles_per_head, seed=seed)
+
+
+def with_lengths(d: dict, lengths) -> dict:
+    """The same tensors with an explicit chunk layout: `lengths[b]` lists the
+    chunk lengths of batch element b (they must sum to L). Used for edge-case
+    layouts (one-token chunks, tails of 63/64/65 rows, ...)."""
+    L = d["Q"].shape[2]
+    nmax = max(len(x) for x in lengths)
+    off = np.full((len(lengths), nmax + 1), L, dtype=np.int32)
+    for b, x in enumerate(lengths):
+        x = np.asarray(x, dtype=np.int64)
+        if x.sum() != L or x.min() < 1:
+            raise ValueError("chunk lengths must be >= 1 and sum to L")
+        off[b, 0] = 0
+        off[b, 1:len(x) + 1] = np.cumsum(x)
+    out = dict(d)
+    out["off"] = off
+    out["n_chunks"] = np.array([len(x) for x in lengths], dtype=np.int32)
+    return out

@@ -84,3 +84,22 @@ def test_budget_selection_arguments_rejected_on_host(lib):
     assert f(FAKE, FAKE, 1, 4, 2, 8, None, FAKE, 100, None, 0, 4, FAKE, FAKE, FAKE, 1 << 30, None) == INV
     assert f(FAKE, FAKE, 1, 3, 2, 8, FAKE, FAKE, 100, None, 0, 4, FAKE, FAKE, FAKE, 1 << 30, None) == INV
     assert f(FAKE, FAKE, 1, 4, 2, 8, FAKE, FAKE, 100, None, 0, 4, FAKE, FAKE, None, 0, None) == WS
+
+
+def test_tile_policy_arguments_rejected_on_host(lib):
+    INV, WS = 1, 5
+    ws = lib.dhsa_sparse_attn_tiles_workspace_size
+    B, Hq, L, nmax = 1, 32, 131072, 823
+    # policy 0 is the plain entry; policy 1 adds one short tile per (b, hq, chunk),
+    # policy 2 has 64-row tiles only
+    assert ws(B, Hq, L, nmax, 0) == lib.dhsa_sparse_attn_workspace_size(B, Hq, L, nmax)
+    assert ws(B, Hq, L, nmax, 1) == ws(B, Hq, L, nmax, 0) + 16 * B * Hq * nmax
+    assert ws(B, Hq, L, nmax, 2) == 256 + 16 * B * Hq * (nmax + L // 64)
+    assert ws(B, Hq, L, nmax, 3) == 0 and ws(B, Hq, L, nmax, -1) == 0
+    f = lib.dhsa_sparse_attn_fwd_tiles
+    args = [FAKE, FAKE, FAKE, 1, 2, 1, 256, 128, FAKE, FAKE, 4, FAKE, FAKE, ctypes.c_float(0.1)]
+    big = ws(1, 2, 256, 4, 2)
+    assert f(*args, 3, FAKE, FAKE, big, None) == INV
+    assert f(*args, -1, FAKE, FAKE, big, None) == INV
+    assert f(*args, 2, FAKE, FAKE, ws(1, 2, 256, 4, 2) - 16, None) == WS
+    assert f(*args, 1, FAKE, None, big, None) == WS

@@ -65,7 +65,7 @@ def test_noalloc_matches_workspace_entry_on_two_calls():
 def test_noalloc_rejects_problems_beyond_static_scratch():
     from long_context_prefill_dhsa_b200 import binding
     lib = binding.load()
-    # 256 + 16 * B*Hq*(Nmax + ceil(L/128)) > 4 MiB for this shape; refused on the host
+    # the workspace size query reports more than 4 MiB for this shape; refused on the host
     B, Hq, Hkv, L, nmax = 1, 64, 8, 131072, 4096
     fake = ctypes.c_void_p(1 << 20)
     st = lib.dhsa_sparse_attn_fwd_noalloc(fake, fake, fake, B, Hq, Hkv, L, 128, fake, fake, nmax, fake, fake,
