@@ -39,6 +39,12 @@
 //   softmax warps.
 // * Pipelines: Q double-buffered; separate K and V rings of 2 stages; a K
 //   stage is released as soon as its QK^T completes, a V stage after its PV.
+//   The producers walk a tile's key stream in registers before they wait for
+//   its stage, so the copies go out right after the wait (the K stage's
+//   barrier gets its byte count first and the producer's arrive last, after
+//   the bias block and tile descriptor are written): the K producer is on
+//   the kernel's critical path, and a few dozen more instructions per tile
+//   there cost several percent.
 //   With two issuing threads the tensor pipe keeps work queued while either
 //   one waits on a barrier.
 // * TMEM (512 columns): three S buffers (3 x 128 fp32 columns) and the O
@@ -390,26 +396,22 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_fwd_kernel(const __gr
       bool ok = true;
       for (int kt = 0; kt < M.T; ++kt, ++g) {
         const int stk = g % NSK, stv = g % NSV, tk = g % NTOK;
-        if (kprod) {
-          // the K stage (and its bias block) of tile g - NSK is free once that QK^T is done
-          if (g >= NSK && !fl.wait(bar(B_SFULL + (g - NSK) % NSB), ((g - NSK) / NSB) & 1)) { ok = false; break; }
-          if (g >= NTOK && !fl.wait(bar(B_TOKEMPTY + tk), ((g / NTOK) - 1) & 1)) { ok = false; break; }
-        } else {
-          // the V stage of tile g - NSV is free once that PV is done
-          if (g >= NSV && !fl.wait(bar(B_PVDONE + (g - NSV) % NSB), ((g - NSV) / NSB) & 1)) { ok = false; break; }
-        }
-        unsigned char* bias = smem + OFF_BIAS + stk * kBiasBytes;
-        // walk the key stream: lane b holds the b-th TMA box of this tile
+        // walk the key stream of this tile first, in registers only (the
+        // stage waits below then overlap it): lane b holds the b-th TMA box,
+        // and bit i of kept the state of slot lane + 32 i
         int slot = 0, causal = 0, d_slot = 0, d_off = 0, nbox = 0, my_y = 0, my_so = 0, my_bx = 0;
-        uint32_t bytes = 0;
+        uint32_t bytes = 0, kept = 0;
         while (slot < BN && sq < M.nseg) {
           const int2 dsc = desc(sq);
           const int rows = min(dsc.y - seg_pos, BN - slot);
           const int groups = (rows + 7) >> 3;
           const int tok0 = dsc.x + seg_pos;
           if (kprod) {
-            for (int s = lane; s < groups * 8; s += 32)
-              *reinterpret_cast<uint16_t*>(bias + noswz_off(slot + s, 0)) = s < rows ? 0 : kBf16NegInf;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const int s = lane + 32 * q;
+              if (s >= slot && s < slot + rows) kept |= 1u << q;
+            }
             if (sq == M.nseg - 1 && tok0 + rows - 1 > M.q0) {
               // diagonal keys past the first query: the piece is the tile's
               // last, slot s >= d_slot holds token s - d_off
@@ -435,22 +437,32 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_fwd_kernel(const __gr
           }
         }
         if (kprod) {
-          for (int s = slot + lane; s < BN; s += 32)
-            *reinterpret_cast<uint16_t*>(bias + noswz_off(s, 0)) = kBf16NegInf;
-          if (lane == 0) tile_info[tk] = make_int4(causal, d_slot, d_off, 0);
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) {
-            mbar_arrive(bar(B_TOKFULL + tk));
-            mbar_arrive_expect_tx(bar(B_KFULL + stk), bytes);
-          }
+          // the K stage (and its bias block) of tile g - NSK is free once that QK^T is done
+          if (g >= NSK && !fl.wait(bar(B_SFULL + (g - NSK) % NSB), ((g - NSK) / NSB) & 1)) { ok = false; break; }
+          if (g >= NTOK && !fl.wait(bar(B_TOKEMPTY + tk), ((g / NTOK) - 1) & 1)) { ok = false; break; }
+          // copies first; the bias block and the tile descriptor follow, and
+          // the stage's barrier completes only after this warp's arrive
+          if (lane == 0) mbar_expect_tx(bar(B_KFULL + stk), bytes);
           __syncwarp();
           const uint32_t dk = sbase + OFF_K + stk * kTileBytes;
           if (lane < nbox) {
             tma_load_2d(dk + my_so, &maps.k[my_bx], bar(B_KFULL + stk), 0, my_y);
             tma_load_2d(dk + kHalfBytes + my_so, &maps.k[my_bx], bar(B_KFULL + stk), 64, my_y);
           }
+          unsigned char* bias = smem + OFF_BIAS + stk * kBiasBytes;
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            *reinterpret_cast<uint16_t*>(bias + noswz_off(lane + 32 * q, 0)) = ((kept >> q) & 1u) ? 0 : kBf16NegInf;
+          if (lane == 0) tile_info[tk] = make_int4(causal, d_slot, d_off, 0);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive(bar(B_TOKFULL + tk));
+            mbar_arrive(bar(B_KFULL + stk));
+          }
         } else {
+          // the V stage of tile g - NSV is free once that PV is done
+          if (g >= NSV && !fl.wait(bar(B_PVDONE + (g - NSV) % NSB), ((g - NSV) / NSB) & 1)) { ok = false; break; }
           if (lane == 0) mbar_arrive_expect_tx(bar(B_VFULL + stv), bytes);
           __syncwarp();
           const uint32_t dv = sbase + OFF_V + stv * kTileBytes;
