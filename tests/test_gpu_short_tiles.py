@@ -114,3 +114,38 @@ def test_column_max_rises_after_first_tile(lib, short_tiles):
     mx, mean = P.compare_out(O, ora.attn_dense(Q, Kf, V))
     print(f"max_abs={mx:.3e} mean_abs={mean:.3e}")
     assert mx <= P.MAX_ABS and mean <= P.MEAN_ABS
+
+
+@needs_gpu
+def test_full_size_128k_tails_on_short_kernel(lib):
+    # the 128K layer in the benchmark's configuration with chunk tails of at
+    # most 64 rows on the short-tile kernel: sampled chunks (a third of them
+    # with such tails) against the fp32 oracle over the GPU's selection, and
+    # the whole output against the 128-row policy
+    w = I.WORKLOADS["llama8b-128k"]
+    d = I.make_inputs(w)
+    layer0, O0 = _run(lib, d, w.k, 0)
+    O0 = O0.clone()
+    layer, O = _run(lib, d, w.k, 1)
+    diff = (O0.float() - O.float()).abs()
+    assert diff.max().item() <= 1e-2 and diff.mean().item() <= 1e-4
+    off, nc = d["off"], d["n_chunks"]
+    sel_gpu = P.gpu_sel_rows(layer.sel, layer.n_sel)
+    n = int(nc[0])
+    lens = np.diff(off[0, : n + 1])
+    tails = np.where((lens % 128 != 0) & (lens % 128 <= 64))[0]
+    rng = np.random.default_rng(11)
+    pick = sorted(set(rng.choice(tails, size=8, replace=False).tolist()) | set(rng.choice(n, size=16, replace=False).tolist()))
+    errs = []
+    for hq in (0, w.Hq - 1):
+        hkv = hq // w.G
+        Qf = ora.bf16_to_f64(d["Q"][0, hq]).astype(np.float32)
+        Kf = ora.bf16_to_f64(d["K"][0, hkv]).astype(np.float32)
+        Vf = ora.bf16_to_f64(d["V"][0, hkv]).astype(np.float32)
+        for i in pick:
+            s, e = int(off[0, i]), int(off[0, i + 1])
+            ref = ora.attn_chunk(Qf, Kf, Vf, off[0], sel_gpu[0][hq][i], i, P.scale(), np.float32)
+            errs.append(np.abs(O[0, hq, s:e].float().cpu().numpy() - ref).ravel())
+    err = np.concatenate(errs)
+    print(f"128K tails on the short kernel: max_abs={err.max():.3e} mean_abs={err.mean():.3e}")
+    assert err.max() <= P.MAX_ABS and err.mean() <= P.MEAN_ABS
