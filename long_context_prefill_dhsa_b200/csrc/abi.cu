@@ -106,7 +106,7 @@ const char* dhsa_status_string(int status) {
 
 int dhsa_last_cuda_error(void) { return t_last_cuda_error; }
 
-int dhsa_version(void) { return 100; }
+int dhsa_version(void) { return 200; }   // 0.2.0: pooling of Q and K in one call, budget selection, query-tile policy
 
 int dhsa_check_device_status(void* stream, uint32_t* device_flags) {
   if (device_flags) *device_flags = 0;
