@@ -63,6 +63,8 @@ def parse():
     # query-tile policy of the attention: 0 = 128-row tiles (default, fastest);
     # 1 = chunk tails of at most 64 rows on the 64-row kernel; 2 = 64-row tiles only
     ap.add_argument("--short-tiles", type=int, default=0, choices=[0, 1, 2])
+    # pooling and the top-k selection as one cooperative launch (top-k rule only)
+    ap.add_argument("--fused-routing", action="store_true")
     return ap.parse_args()
 
 
@@ -332,13 +334,13 @@ def main():
     k_sel, bud, recent, sel_desc = selection_rule(args, w, d["off"].shape[1] - 1)
     bud_arg = torch.from_numpy(bud).to(dev) if isinstance(bud, np.ndarray) else bud
     layer = binding.DHSAPrefill(w.B, w.Hq, w.Hkv, w.L, off, nc, k_sel, device=dev, budget=bud_arg, recent=recent,
-                                short_tiles=args.short_tiles)
+                                short_tiles=args.short_tiles, fused_routing=args.fused_routing)
     stream = torch.cuda.current_stream()
 
     ev = lambda: torch.cuda.Event(enable_timing=True)
     # pool (Q and K), key norms + score tiles + select, CSR scan + fill, work list + attention
     # (tile policy 1 launches both attention kernels)
-    n_launch_per_step = 8 + (1 if args.short_tiles == 1 else 0)
+    n_launch_per_step = 8 + (1 if args.short_tiles == 1 else 0) - (3 if args.fused_routing else 0)
 
     def step(timed_stages=None):
         if timed_stages is None:
@@ -457,6 +459,8 @@ def main():
                        "k": w.k, "selection": sel_desc,
                        "query_tiles": ["128 rows", "128 rows, tails <= 64 rows on the 64-row kernel",
                                        "64 rows"][args.short_tiles],
+                       "routing_launches": "fused (one cooperative launch up to the selection)"
+                                           if args.fused_routing else "separate",
                        "chunk_len": f"{w.length_kind}[{w.length_lo},{w.length_hi}]", "n_chunks": nmax,
                        "kept_density": pairs / (w.B * w.Hq * w.L * (w.L + 1) / 2),
                        "parallelism": f"replicas x{world} (independent layers, no collective)",

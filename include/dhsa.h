@@ -168,6 +168,27 @@ int dhsa_chunk_score_select_budget(const float* Qp, const float* Kp, int B, int 
                                    void* workspace, size_t workspace_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * 2c. Pooling, similarity and top-k in one launch.
+ *    Sources as for 1. and 2.; the gist.science technical summary places the
+ *    routing module right after the Q/K projections, so it runs as one unit.
+ *
+ *    Does what dhsa_chunk_pool_qk followed by dhsa_chunk_score_topk do, with
+ *    the same results bit for bit, as one cooperative launch: pooling of Q
+ *    and K, key norms and score tiles, then the selection, separated by
+ *    grid-wide barriers (each bounded: a barrier that waits more than 1 s
+ *    sets DHSA_DEVFLAG_WAIT_TIMEOUT). Arguments and layouts are those of the
+ *    two calls; Qp and Kp are written as by 1b.
+ *    workspace: dhsa_route_fused_workspace_size(B, Hq, Nmax) bytes (equal to
+ *    dhsa_score_topk_workspace_size; its first 4 bytes hold the barrier
+ *    count, reset by this call on `stream`). Calls sharing a workspace must
+ *    not overlap on the GPU.
+ * ------------------------------------------------------------------------- */
+size_t dhsa_route_fused_workspace_size(int B, int Hq, int Nmax);
+int dhsa_route_fused(const void* Q, const void* K, int B, int Hq, int Hkv, int L, int head_dim, const int32_t* off,
+                     const int32_t* n_chunks, int Nmax, int k, float* Qp, float* Kp, int32_t* sel, int32_t* n_sel,
+                     void* workspace, size_t workspace_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
  * 3. Upsampling to the token keep-set, stored as a block CSR.
  *    Source: OpenReview abstract (chunk scores are upsampled to the token
  *    level to decide which token interactions are kept); gist.science

@@ -52,6 +52,8 @@ _SIGNATURES = {
     "dhsa_chunk_score_topk": (_I, [_P, _P, _I, _I, _I, _I, _P, _I, _P, _P, _P, _SZ, _P]),
     "dhsa_budget_max_chunks": (_I, []),
     "dhsa_chunk_score_select_budget": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, _I, _P, _I, _I, _P, _P, _P, _SZ, _P]),
+    "dhsa_route_fused_workspace_size": (_SZ, [_I, _I, _I]),
+    "dhsa_route_fused": (_I, [_P, _P, _I, _I, _I, _I, _I, _P, _P, _I, _I, _P, _P, _P, _P, _P, _SZ, _P]),
     "dhsa_csr_nnz_upper": (_SZ, [_I, _I, _I, _I]),
     "dhsa_build_block_csr": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P]),
     "dhsa_sparse_attn_workspace_size": (_SZ, [_I, _I, _I, _I]),
@@ -198,6 +200,43 @@ def chunk_score_topk(Qp: torch.Tensor, Kp: torch.Tensor, n_chunks: torch.Tensor,
     return sel, n_sel
 
 
+def route_fused(Q: torch.Tensor, K: torch.Tensor, off: torch.Tensor, n_chunks: torch.Tensor, k: int,
+                Qp: Optional[torch.Tensor] = None, Kp: Optional[torch.Tensor] = None,
+                sel: Optional[torch.Tensor] = None, n_sel: Optional[torch.Tensor] = None,
+                workspace: Optional[torch.Tensor] = None):
+    """Pooling of Q and K plus the top-k selection in one launch (include/dhsa.h,
+    2c); the same results as chunk_pool_qk followed by chunk_score_topk.
+    Returns (Qp, Kp, sel, n_sel)."""
+    B, Hq, L, d = Q.shape
+    Hkv = K.shape[1]
+    nmax = off.shape[1] - 1
+    _need(Q, torch.bfloat16, None, "Q")
+    _need(K, torch.bfloat16, (B, Hkv, L, d), "K")
+    _need(off, torch.int32, (B, nmax + 1), "off")
+    _need(n_chunks, torch.int32, (B,), "n_chunks")
+    lib = load()
+    stride = lib.dhsa_sel_stride(k, nmax)
+    if Qp is None:
+        Qp = torch.empty((B, Hq, nmax, d), dtype=torch.float32, device=Q.device)
+    if Kp is None:
+        Kp = torch.empty((B, Hkv, nmax, d), dtype=torch.float32, device=Q.device)
+    if sel is None:
+        sel = torch.empty((B, Hq, nmax, stride), dtype=torch.int32, device=Q.device)
+    if n_sel is None:
+        n_sel = torch.empty((B, Hq, nmax), dtype=torch.int32, device=Q.device)
+    _need(Qp, torch.float32, (B, Hq, nmax, d), "Qp")
+    _need(Kp, torch.float32, (B, Hkv, nmax, d), "Kp")
+    _need(sel, torch.int32, (B, Hq, nmax, stride), "sel")
+    _need(n_sel, torch.int32, (B, Hq, nmax), "n_sel")
+    ws_bytes = lib.dhsa_route_fused_workspace_size(B, Hq, nmax)
+    if workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=Q.device)
+    _check(lib.dhsa_route_fused(_ptr(Q), _ptr(K), B, Hq, Hkv, L, d, _ptr(off), _ptr(n_chunks), nmax, k, _ptr(Qp),
+                                _ptr(Kp), _ptr(sel), _ptr(n_sel), _ptr(workspace),
+                                workspace.numel() * workspace.element_size(), _stream_ptr()), "dhsa_route_fused")
+    return Qp, Kp, sel, n_sel
+
+
 def chunk_score_select_budget(Qp: torch.Tensor, Kp: torch.Tensor, off: torch.Tensor, n_chunks: torch.Tensor,
                               budget, recent: int, k_max: int, sel: Optional[torch.Tensor] = None,
                               n_sel: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None):
@@ -318,14 +357,19 @@ class DHSAPrefill:
     a window of `recent` chunks and at most k earlier chunks per row.
     `short_tiles` picks the query-tile policy of the attention (0: 128-row
     tiles only, the fast default; 1 and 2: see sparse_attn_fwd).
+    `fused_routing` runs pooling and the top-k selection as one launch
+    (route_fused; top-k rule only).
     """
 
     def __init__(self, B: int, Hq: int, Hkv: int, L: int, off: torch.Tensor, n_chunks: torch.Tensor, k: int,
                  device="cuda", softmax_scale: Optional[float] = None, budget=None, recent: int = 0,
-                 short_tiles: int = 0):
+                 short_tiles: int = 0, fused_routing: bool = False):
         lib = load()
         self.B, self.Hq, self.Hkv, self.L, self.k = B, Hq, Hkv, L, k
         self.short_tiles = short_tiles
+        if fused_routing and budget is not None:
+            raise ValueError("fused_routing supports the top-k rule only")
+        self.fused_routing = fused_routing
         self.budget, self.recent = budget, recent
         self.off, self.n_chunks = off, n_chunks
         self.nmax = off.shape[1] - 1
@@ -347,6 +391,12 @@ class DHSAPrefill:
         self.O = torch.empty((B, Hq, L, 128), dtype=torch.bfloat16, device=dev)
 
     def routing(self, Q, K):
+        if self.fused_routing:
+            route_fused(Q, K, self.off, self.n_chunks, self.k, Qp=self.Qp, Kp=self.Kp, sel=self.sel,
+                        n_sel=self.n_sel, workspace=self.ws_topk)
+            build_block_csr(self.sel, self.n_sel, self.k, self.off, self.n_chunks, row_ptr=self.row_ptr,
+                            col_idx=self.col_idx, cost=self.cost)
+            return
         chunk_pool_qk(Q, K, self.off, self.n_chunks, Qp=self.Qp, Kp=self.Kp)
         if self.budget is None:
             chunk_score_topk(self.Qp, self.Kp, self.n_chunks, self.k, sel=self.sel, n_sel=self.n_sel,

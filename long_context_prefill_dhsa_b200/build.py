@@ -20,7 +20,7 @@ CSRC = os.path.join(PKG, "csrc")
 OBJ = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libdhsa.so")
 SOURCES = ["abi.cu", "pool.cu", "score_topk.cu", "csr.cu", "items.cu", "attn.cu", "attn_fwd.cu", "attn_short.cu"]
-HEADERS = ["common.cuh", "sm100_ptx.cuh", "tmap.cuh"]
+HEADERS = ["common.cuh", "sm100_ptx.cuh", "tmap.cuh", "pool_row.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

@@ -16,6 +16,9 @@ int score_topk_stride(int k, int Nmax);
 size_t score_topk_ws_bytes(int B, int Hq, int Nmax);
 int launch_score_topk(const float* Qp, const float* Kp, int B, int Hq, int Hkv, int Nmax, const int32_t* n_chunks,
                       int k, int32_t* sel, int32_t* n_sel, void* ws, cudaStream_t stream);
+int launch_route_fused(const void* Q, const void* K, int B, int Hq, int Hkv, int L, const int32_t* off,
+                       const int32_t* n_chunks, int Nmax, int k, float* Qp, float* Kp, int32_t* sel, int32_t* n_sel,
+                       void* ws, unsigned int* status, cudaStream_t stream);
 int score_budget_max_chunks();
 int launch_score_budget(const float* Qp, const float* Kp, int B, int Hq, int Hkv, int Nmax, const int32_t* off,
                         const int32_t* n_chunks, int budget, const int32_t* budgets, int recent, int k_max,
@@ -176,6 +179,30 @@ int dhsa_chunk_score_topk(const float* Qp, const float* Kp, int B, int Hq, int H
   if (st != DHSA_OK) return st;
   return launch_score_topk(Qp, Kp, B, Hq, Hkv, Nmax, n_chunks, k, sel, n_sel, need ? workspace : nullptr,
                            static_cast<cudaStream_t>(stream));
+}
+
+size_t dhsa_route_fused_workspace_size(int B, int Hq, int Nmax) {
+  if (B <= 0 || Hq <= 0 || Nmax <= 0) return 0;
+  return score_topk_ws_bytes(B, Hq, Nmax);
+}
+
+int dhsa_route_fused(const void* Q, const void* K, int B, int Hq, int Hkv, int L, int head_dim, const int32_t* off,
+                     const int32_t* n_chunks, int Nmax, int k, float* Qp, float* Kp, int32_t* sel, int32_t* n_sel,
+                     void* workspace, size_t workspace_bytes, void* stream) {
+  int st = check_layout(B, Hq, L, Nmax, off, n_chunks);
+  if (st != DHSA_OK) return st;
+  if (Hkv <= 0 || Hq % Hkv != 0 || k < 0) return DHSA_ERR_INVALID_ARG;
+  if (!Q || !K || !Qp || !Kp || !sel || !n_sel || !aligned16(Q) || !aligned16(K) || !aligned16(Qp) ||
+      !aligned16(Kp))
+    return DHSA_ERR_INVALID_ARG;
+  if (head_dim != kHeadDim) return DHSA_ERR_UNSUPPORTED;
+  const size_t need = score_topk_ws_bytes(B, Hq, Nmax);
+  if (!workspace || workspace_bytes < need || !aligned16(workspace)) return DHSA_ERR_WORKSPACE;
+  if ((st = check_device_sm100()) != DHSA_OK) return st;
+  unsigned int* status = device_status_ptr();
+  if (!status) return DHSA_ERR_CUDA;
+  return launch_route_fused(Q, K, B, Hq, Hkv, L, off, n_chunks, Nmax, k, Qp, Kp, sel, n_sel, workspace, status,
+                            static_cast<cudaStream_t>(stream));
 }
 
 int dhsa_budget_max_chunks(void) { return score_budget_max_chunks(); }

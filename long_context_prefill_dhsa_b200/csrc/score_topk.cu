@@ -24,6 +24,8 @@
 //      lower index). The kept indices are written ascending, diagonal last.
 // For very many chunks the workspace is processed in batches of heads.
 #include "common.cuh"
+#include "pool_row.cuh"
+#include "sm100_ptx.cuh"
 
 namespace dhsa {
 namespace {
@@ -50,11 +52,9 @@ __device__ __forceinline__ unsigned lanemask_lt() {
 __host__ __device__ __forceinline__ long long tri(long long i) { return i * (i - 1) / 2; }
 
 // ------------------------------------------------------------------ 1. key norms
-__global__ void __launch_bounds__(256) key_norm_kernel(const float* __restrict__ Kp, long long rows,
-                                                       float* __restrict__ kn) {
-  const long long r = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+// one warp: the norm of pooled key row r
+__device__ __forceinline__ void key_norm_row(const float* __restrict__ Kp, long long r, float* __restrict__ kn) {
   const int lane = threadIdx.x & 31;
-  if (r >= rows) return;
   const float4 v = reinterpret_cast<const float4*>(Kp + r * kHeadDim)[lane];
   double s = (double)v.x * v.x + (double)v.y * v.y + (double)v.z * v.z + (double)v.w * v.w;
 #pragma unroll
@@ -62,16 +62,21 @@ __global__ void __launch_bounds__(256) key_norm_kernel(const float* __restrict__
   if (lane == 0) kn[r] = (float)(sqrt(s) * (1.0 + 1e-6));   // fp32 rounding covered by the margin
 }
 
+__global__ void __launch_bounds__(256) key_norm_kernel(const float* __restrict__ Kp, long long rows,
+                                                       float* __restrict__ kn) {
+  const long long r = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  if (r < rows) key_norm_row(Kp, r, kn);
+}
+
 // ------------------------------------------------------------------ 2. fp32 score tiles
-__global__ void __launch_bounds__(256, 2) score_tile_kernel(const float* __restrict__ Qp,
-                                                         const float* __restrict__ Kp, int Hq, int G, int Nmax,
-                                                         const int32_t* __restrict__ n_chunks, long long bh0,
-                                                         int n_rb, int n_kb, float* __restrict__ ws) {
-  extern __shared__ __align__(16) float sm[];
+// one block: score tile (rb, kb) of head bh0 + bhl into that head's packed
+// rows of ws (sm: TR * 128 + TK * 132 floats of shared memory)
+__device__ __forceinline__ void score_tile_body(const float* __restrict__ Qp, const float* __restrict__ Kp, int Hq,
+                                                int G, int Nmax, const int32_t* __restrict__ n_chunks, long long bh0,
+                                                int bhl, int rb, int kb, float* __restrict__ ws, float* sm) {
   float* Qs = sm;                        // [TR][128]
   float* Ks = sm + TR * kHeadDim;        // [TK][132]
-  const int kb = blockIdx.x % n_kb, rb = blockIdx.x / n_kb;
-  const long long bh = bh0 + blockIdx.y;
+  const long long bh = bh0 + bhl;
   const int b = (int)(bh / Hq), hq = (int)(bh % Hq);
   const int n = n_chunks[b];
   const int i0 = rb * TR, j0 = kb * TK;
@@ -116,7 +121,7 @@ __global__ void __launch_bounds__(256, 2) score_tile_kernel(const float* __restr
       }
     }
   }
-  float* head = ws + blockIdx.y * tri(Nmax);
+  float* head = ws + bhl * tri(Nmax);
 #pragma unroll
   for (int r = 0; r < 8; ++r) {
     const int i = i0 + warp * 8 + r;
@@ -127,6 +132,14 @@ __global__ void __launch_bounds__(256, 2) score_tile_kernel(const float* __restr
       if (j < i) head[tri(i) + j] = acc[r][c];
     }
   }
+}
+
+__global__ void __launch_bounds__(256, 2) score_tile_kernel(const float* __restrict__ Qp,
+                                                         const float* __restrict__ Kp, int Hq, int G, int Nmax,
+                                                         const int32_t* __restrict__ n_chunks, long long bh0,
+                                                         int n_rb, int n_kb, float* __restrict__ ws) {
+  extern __shared__ __align__(16) float sm[];
+  score_tile_body(Qp, Kp, Hq, G, Nmax, n_chunks, bh0, blockIdx.y, blockIdx.x / n_kb, blockIdx.x % n_kb, ws, sm);
 }
 
 // ------------------------------------------------------------------ 3. selection
@@ -326,17 +339,15 @@ __device__ __forceinline__ bool in_cut(const Cut& cut, float s32, int j, const f
   return cut.all_band || !ranks_above(cut.cutE, cut.cutJ, exact_score(qrow, Kp + (kv_row0 + j) * kHeadDim), j);
 }
 
-__global__ void __launch_bounds__(256) select_kernel(const float* __restrict__ Qp, const float* __restrict__ Kp,
-                                                     const float* __restrict__ kn, int Hq, int G, int Nmax,
-                                                     const int32_t* __restrict__ n_chunks, int k, int stride,
-                                                     long long bh0, long long n_rows,
-                                                     const float* __restrict__ ws, int32_t* __restrict__ sel,
-                                                     int32_t* __restrict__ n_sel) {
-  __shared__ int hist_all[8][256];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+// one warp: the top-k row wr of the head batch starting at head bh0 (hist:
+// this warp's 256 ints of shared scratch)
+__device__ __forceinline__ void select_row(const float* __restrict__ Qp, const float* __restrict__ Kp,
+                                           const float* __restrict__ kn, int Hq, int G, int Nmax,
+                                           const int32_t* __restrict__ n_chunks, int k, int stride, long long bh0,
+                                           long long wr, const float* __restrict__ ws, int32_t* __restrict__ sel,
+                                           int32_t* __restrict__ n_sel, int* hist) {
+  const int lane = threadIdx.x & 31;
   const unsigned full = 0xffffffffu;
-  const long long wr = (long long)blockIdx.x * 8 + warp;      // row within the head batch
-  if (wr >= n_rows) return;
   const long long bhl = wr / Nmax;
   const int i = (int)(wr % Nmax);
   const long long bh = bh0 + bhl;
@@ -353,7 +364,7 @@ __global__ void __launch_bounds__(256) select_kernel(const float* __restrict__ Q
       const float* row = ws + bhl * tri(Nmax) + tri(i);
       const long long kv_row0 = ((long long)b * (Hq / G) + hq / G) * Nmax;
       const float* qrow = Qp + (bh * Nmax + i) * kHeadDim;
-      const Cut cut = topm_cut(row, i, m, hist_all[warp], qrow, Kp, kv_row0, kn);
+      const Cut cut = topm_cut(row, i, m, hist, qrow, Kp, kv_row0, kn);
       // --- output, ascending
       int written = 0;
       for (int j0 = 0; j0 < i; j0 += 32) {
@@ -371,6 +382,18 @@ __global__ void __launch_bounds__(256) select_kernel(const float* __restrict__ Q
   }
   for (int q = cnt + lane; q < stride; q += 32) out[q] = -1;
   if (lane == 0) n_sel[bh * Nmax + i] = cnt;
+}
+
+__global__ void __launch_bounds__(256) select_kernel(const float* __restrict__ Qp, const float* __restrict__ Kp,
+                                                     const float* __restrict__ kn, int Hq, int G, int Nmax,
+                                                     const int32_t* __restrict__ n_chunks, int k, int stride,
+                                                     long long bh0, long long n_rows,
+                                                     const float* __restrict__ ws, int32_t* __restrict__ sel,
+                                                     int32_t* __restrict__ n_sel) {
+  __shared__ int hist_all[8][256];
+  const int warp = threadIdx.x >> 5;
+  const long long wr = (long long)blockIdx.x * 8 + warp;      // row within the head batch
+  if (wr < n_rows) select_row(Qp, Kp, kn, Hq, G, Nmax, n_chunks, k, stride, bh0, wr, ws, sel, n_sel, hist_all[warp]);
 }
 
 // ------------------------------------------------------------------ 3'. row budgets
@@ -489,6 +512,84 @@ long long heads_per_batch(int B, int Hq, int Nmax) {
   return h;
 }
 
+// ------------------------------------------------------------------ 4. fused routing
+// Pooling of Q and K, key norms, score tiles and the top-k selection in one
+// cooperative launch, with a grid-wide barrier between the phases that read
+// what the previous one wrote. Each phase runs the same per-warp or
+// per-block code as its separate kernel, so the results are bit-identical.
+struct GridBar {
+  unsigned int* count;    // arrivals so far (zeroed before the launch)
+  unsigned int* status;
+};
+
+__device__ __forceinline__ unsigned ld_acquire_u32(const unsigned int* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Every block arrives once per barrier; thread 0 waits until all have, and
+// gives up after 1 s of wall-clock time (DHSA_DEVFLAG_WAIT_TIMEOUT).
+__device__ __forceinline__ void grid_barrier(const GridBar& gb, unsigned& phase) {
+  __syncthreads();
+  ++phase;
+  if (threadIdx.x == 0) {
+    __threadfence();
+    atomicAdd(gb.count, 1u);
+    const unsigned target = phase * gridDim.x;
+    const uint64_t t0 = ptx::globaltimer_ns();
+    while (ld_acquire_u32(gb.count) < target) {
+      if (ptx::globaltimer_ns() - t0 > 1000000000ull) {
+        raise_device_flag(gb.status, DHSA_DEVFLAG_WAIT_TIMEOUT);
+        break;
+      }
+      __nanosleep(64);
+    }
+    __threadfence();
+  }
+  __syncthreads();
+}
+
+__global__ void __launch_bounds__(256, 2) route_fused_kernel(const uint4* __restrict__ Q, const uint4* __restrict__ K,
+                                                          int B, int Hq, int Hkv, int L,
+                                                          const int32_t* __restrict__ off,
+                                                          const int32_t* __restrict__ n_chunks, int Nmax, int k,
+                                                          int stride, long long hb, float* __restrict__ Qp,
+                                                          float* __restrict__ Kp, float* __restrict__ kn,
+                                                          float* __restrict__ scores, int32_t* __restrict__ sel,
+                                                          int32_t* __restrict__ n_sel, GridBar gb) {
+  extern __shared__ __align__(16) float sm[];
+  const int G = Hq / Hkv;
+  const long long gwarp = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const long long nwarps = (long long)gridDim.x * (blockDim.x >> 5);
+  unsigned phase = 0;
+  // pooled Q and K rows
+  const long long rows_q = (long long)B * Hq * Nmax, rows_k = (long long)B * Hkv * Nmax;
+  for (long long w = gwarp; w < rows_q + rows_k; w += nwarps) {
+    if (w < rows_q) pool_row(Q, Hq, L, off, n_chunks, Nmax, w, Qp);
+    else pool_row(K, Hkv, L, off, n_chunks, Nmax, w - rows_q, Kp);
+  }
+  grid_barrier(gb, phase);
+  // key norms (read by the selection only) and the score tiles of each head batch
+  for (long long r = gwarp; r < rows_k; r += nwarps) key_norm_row(Kp, r, kn);
+  const int n_rb = (Nmax + TR - 1) / TR, n_kb = (Nmax + TK - 1) / TK;
+  const long long total = (long long)B * Hq;
+  int* hist = reinterpret_cast<int*>(sm) + (threadIdx.x >> 5) * 256;
+  for (long long h0 = 0; h0 < total; h0 += hb) {
+    const long long nh = total - h0 < hb ? total - h0 : hb;
+    const long long tiles = nh * n_rb * n_kb;
+    for (long long t = blockIdx.x; t < tiles; t += gridDim.x) {
+      const int bhl = (int)(t / (n_rb * n_kb)), rest = (int)(t % (n_rb * n_kb));
+      score_tile_body(Qp, Kp, Hq, G, Nmax, n_chunks, h0, bhl, rest / n_kb, rest % n_kb, scores, sm);
+      __syncthreads();   // the next tile restages shared memory
+    }
+    grid_barrier(gb, phase);
+    for (long long wr = gwarp; wr < nh * Nmax; wr += nwarps)
+      select_row(Qp, Kp, kn, Hq, G, Nmax, n_chunks, k, stride, h0, wr, scores, sel, n_sel, hist);
+    if (h0 + hb < total) grid_barrier(gb, phase);   // the next head batch overwrites the scores
+  }
+}
+
 }  // namespace
 
 int score_topk_stride(int k, int Nmax) { return (k < Nmax - 1 ? k : Nmax - 1) + 1; }
@@ -527,6 +628,37 @@ int launch_score_topk(const float* Qp, const float* Kp, int B, int Hq, int Hkv, 
     if ((st = launch_status()) != DHSA_OK) return st;
   }
   return DHSA_OK;
+}
+
+// All of routing up to the selection in one cooperative launch (workspace as
+// for launch_score_topk; its first 4 bytes hold the grid barrier's counter).
+int launch_route_fused(const void* Q, const void* K, int B, int Hq, int Hkv, int L, const int32_t* off,
+                       const int32_t* n_chunks, int Nmax, int k, float* Qp, float* Kp, int32_t* sel, int32_t* n_sel,
+                       void* ws, unsigned int* status, cudaStream_t stream) {
+  const int stride = score_topk_stride(k, Nmax);
+  float* kn = reinterpret_cast<float*>(static_cast<char*>(ws) + 256);
+  const size_t kn_bytes = (sizeof(float) * (size_t)B * Hq * Nmax + 255) & ~size_t(255);
+  float* scores = reinterpret_cast<float*>(static_cast<char*>(ws) + 256 + kn_bytes);
+  const long long hb = heads_per_batch(B, Hq, Nmax);
+  const int smem = (int)(sizeof(float) * (TR * kHeadDim + TK * kKsStride));
+  cudaError_t e = cudaFuncSetAttribute(route_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  int dev = 0, sms = 0, per_sm = 0;
+  if (e == cudaSuccess) e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, route_fused_kernel, 256, smem);
+  if (e == cudaSuccess) e = cudaMemsetAsync(ws, 0, sizeof(unsigned int), stream);
+  if (e != cudaSuccess) return cuda_status(e);
+  if (per_sm < 1) return DHSA_ERR_UNSUPPORTED;
+  GridBar gb{static_cast<unsigned int*>(ws), status};
+  const uint4* q4 = static_cast<const uint4*>(Q);
+  const uint4* k4 = static_cast<const uint4*>(K);
+  void* args[] = {(void*)&q4,     (void*)&k4,   (void*)&B,     (void*)&Hq,   (void*)&Hkv,   (void*)&L,
+                  (void*)&off,    (void*)&n_chunks, (void*)&Nmax, (void*)&k, (void*)&stride, (void*)&hb,
+                  (void*)&Qp,     (void*)&Kp,   (void*)&kn,    (void*)&scores, (void*)&sel, (void*)&n_sel,
+                  (void*)&gb};
+  e = cudaLaunchCooperativeKernel((const void*)route_fused_kernel, dim3(per_sm * sms), dim3(256), args, (size_t)smem,
+                                  stream);
+  return cuda_status(e);
 }
 
 int score_budget_max_chunks() { return kBudgetCap - 1; }

@@ -103,3 +103,18 @@ def test_tile_policy_arguments_rejected_on_host(lib):
     assert f(*args, -1, FAKE, FAKE, big, None) == INV
     assert f(*args, 2, FAKE, FAKE, ws(1, 2, 256, 4, 2) - 16, None) == WS
     assert f(*args, 1, FAKE, None, big, None) == WS
+
+
+def test_fused_routing_arguments_rejected_on_host(lib):
+    INV, UNS, WS = 1, 2, 5
+    f = lib.dhsa_route_fused
+    ws = lib.dhsa_route_fused_workspace_size(1, 4, 8)
+    assert ws == lib.dhsa_score_topk_workspace_size(1, 4, 8) and ws >= 256
+    #          Q     K     B  Hq Hkv  L  hd  off   n_ch Nmax k  Qp    Kp    sel   n_sel ws    bytes stream
+    assert f(FAKE, FAKE, 1, 4, 2, 64, 128, FAKE, FAKE, 8, -1, FAKE, FAKE, FAKE, FAKE, FAKE, ws, None) == INV
+    assert f(FAKE, FAKE, 1, 3, 2, 64, 128, FAKE, FAKE, 8, 2, FAKE, FAKE, FAKE, FAKE, FAKE, ws, None) == INV
+    assert f(None, FAKE, 1, 4, 2, 64, 128, FAKE, FAKE, 8, 2, FAKE, FAKE, FAKE, FAKE, FAKE, ws, None) == INV
+    assert f(FAKE, FAKE, 1, 4, 2, 64, 128, FAKE, FAKE, 8, 2, FAKE, FAKE, None, FAKE, FAKE, ws, None) == INV
+    assert f(FAKE, FAKE, 1, 4, 2, 64, 96, FAKE, FAKE, 8, 2, FAKE, FAKE, FAKE, FAKE, FAKE, ws, None) == UNS
+    assert f(FAKE, FAKE, 1, 4, 2, 64, 128, FAKE, FAKE, 8, 2, FAKE, FAKE, FAKE, FAKE, None, ws, None) == WS
+    assert f(FAKE, FAKE, 1, 4, 2, 64, 128, FAKE, FAKE, 8, 2, FAKE, FAKE, FAKE, FAKE, FAKE, ws - 16, None) == WS
