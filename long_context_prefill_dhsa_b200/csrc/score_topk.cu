@@ -70,16 +70,19 @@ __global__ void __launch_bounds__(256) key_norm_kernel(const float* __restrict__
 
 // ------------------------------------------------------------------ 2. fp32 score tiles
 // one block: score tile (rb, kb) of head bh0 + bhl into that head's packed
-// rows of ws (sm: TR * 128 + TK * 132 floats of shared memory)
+// rows of ws; a tile is TR query rows x 32 * KC keys (sm: TR * 128 +
+// 32 * KC * 132 floats of shared memory). Every score is one thread's fp32
+// dot product in a fixed order, whatever KC.
+template <int KC>
 __device__ __forceinline__ void score_tile_body(const float* __restrict__ Qp, const float* __restrict__ Kp, int Hq,
                                                 int G, int Nmax, const int32_t* __restrict__ n_chunks, long long bh0,
                                                 int bhl, int rb, int kb, float* __restrict__ ws, float* sm) {
   float* Qs = sm;                        // [TR][128]
-  float* Ks = sm + TR * kHeadDim;        // [TK][132]
+  float* Ks = sm + TR * kHeadDim;        // [32 * KC][132]
   const long long bh = bh0 + bhl;
   const int b = (int)(bh / Hq), hq = (int)(bh % Hq);
   const int n = n_chunks[b];
-  const int i0 = rb * TR, j0 = kb * TK;
+  const int i0 = rb * TR, j0 = kb * 32 * KC;
   const int i_hi = min(i0 + TR, n);                 // rows [i0, i_hi)
   if (i0 >= n || j0 >= i_hi - 1) return;            // no j < i in this tile
   const long long kv_row0 = ((long long)b * (Hq / G) + hq / G) * Nmax;
@@ -90,7 +93,7 @@ __device__ __forceinline__ void score_tile_body(const float* __restrict__ Qp, co
     if (i < n) v = reinterpret_cast<const float4*>(Qp + (bh * Nmax + i) * kHeadDim)[c4];
     reinterpret_cast<float4*>(Qs + r * kHeadDim)[c4] = v;
   }
-  for (int idx = threadIdx.x; idx < TK * 32; idx += blockDim.x) {
+  for (int idx = threadIdx.x; idx < 32 * KC * 32; idx += blockDim.x) {
     const int r = idx >> 5, c4 = idx & 31;
     const int j = j0 + r;
     float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -99,21 +102,21 @@ __device__ __forceinline__ void score_tile_body(const float* __restrict__ Qp, co
   }
   __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  float acc[8][4];
+  float acc[8][KC];
 #pragma unroll
   for (int r = 0; r < 8; ++r)
 #pragma unroll
-    for (int c = 0; c < 4; ++c) acc[r][c] = 0.f;
+    for (int c = 0; c < KC; ++c) acc[r][c] = 0.f;
 #pragma unroll 2
   for (int d = 0; d < kHeadDim; d += 4) {
-    float4 kv[4];
+    float4 kv[KC];
 #pragma unroll
-    for (int c = 0; c < 4; ++c) kv[c] = *reinterpret_cast<const float4*>(Ks + (lane + 32 * c) * kKsStride + d);
+    for (int c = 0; c < KC; ++c) kv[c] = *reinterpret_cast<const float4*>(Ks + (lane + 32 * c) * kKsStride + d);
 #pragma unroll
     for (int r = 0; r < 8; ++r) {
       const float4 qv = *reinterpret_cast<const float4*>(Qs + (warp * 8 + r) * kHeadDim + d);
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < KC; ++c) {
         acc[r][c] = fmaf(qv.x, kv[c].x, acc[r][c]);
         acc[r][c] = fmaf(qv.y, kv[c].y, acc[r][c]);
         acc[r][c] = fmaf(qv.z, kv[c].z, acc[r][c]);
@@ -127,7 +130,7 @@ __device__ __forceinline__ void score_tile_body(const float* __restrict__ Qp, co
     const int i = i0 + warp * 8 + r;
     if (i >= i_hi) continue;
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
+    for (int c = 0; c < KC; ++c) {
       const int j = j0 + lane + 32 * c;
       if (j < i) head[tri(i) + j] = acc[r][c];
     }
@@ -139,7 +142,8 @@ __global__ void __launch_bounds__(256, 2) score_tile_kernel(const float* __restr
                                                          const int32_t* __restrict__ n_chunks, long long bh0,
                                                          int n_rb, int n_kb, float* __restrict__ ws) {
   extern __shared__ __align__(16) float sm[];
-  score_tile_body(Qp, Kp, Hq, G, Nmax, n_chunks, bh0, blockIdx.y, blockIdx.x / n_kb, blockIdx.x % n_kb, ws, sm);
+  score_tile_body<TK / 32>(Qp, Kp, Hq, G, Nmax, n_chunks, bh0, blockIdx.y, blockIdx.x / n_kb, blockIdx.x % n_kb, ws,
+                          sm);
 }
 
 // ------------------------------------------------------------------ 3. selection
@@ -550,7 +554,9 @@ __device__ __forceinline__ void grid_barrier(const GridBar& gb, unsigned& phase)
   __syncthreads();
 }
 
-__global__ void __launch_bounds__(256, 2) route_fused_kernel(const uint4* __restrict__ Q, const uint4* __restrict__ K,
+constexpr int kFusedKC = 2;   // 64-key score tiles in the fused kernel: three blocks per SM
+
+__global__ void __launch_bounds__(256, 3) route_fused_kernel(const uint4* __restrict__ Q, const uint4* __restrict__ K,
                                                           int B, int Hq, int Hkv, int L,
                                                           const int32_t* __restrict__ off,
                                                           const int32_t* __restrict__ n_chunks, int Nmax, int k,
@@ -572,7 +578,7 @@ __global__ void __launch_bounds__(256, 2) route_fused_kernel(const uint4* __rest
   grid_barrier(gb, phase);
   // key norms (read by the selection only) and the score tiles of each head batch
   for (long long r = gwarp; r < rows_k; r += nwarps) key_norm_row(Kp, r, kn);
-  const int n_rb = (Nmax + TR - 1) / TR, n_kb = (Nmax + TK - 1) / TK;
+  const int n_rb = (Nmax + TR - 1) / TR, n_kb = (Nmax + 32 * kFusedKC - 1) / (32 * kFusedKC);
   const long long total = (long long)B * Hq;
   int* hist = reinterpret_cast<int*>(sm) + (threadIdx.x >> 5) * 256;
   for (long long h0 = 0; h0 < total; h0 += hb) {
@@ -580,7 +586,7 @@ __global__ void __launch_bounds__(256, 2) route_fused_kernel(const uint4* __rest
     const long long tiles = nh * n_rb * n_kb;
     for (long long t = blockIdx.x; t < tiles; t += gridDim.x) {
       const int bhl = (int)(t / (n_rb * n_kb)), rest = (int)(t % (n_rb * n_kb));
-      score_tile_body(Qp, Kp, Hq, G, Nmax, n_chunks, h0, bhl, rest / n_kb, rest % n_kb, scores, sm);
+      score_tile_body<kFusedKC>(Qp, Kp, Hq, G, Nmax, n_chunks, h0, bhl, rest / n_kb, rest % n_kb, scores, sm);
       __syncthreads();   // the next tile restages shared memory
     }
     grid_barrier(gb, phase);
@@ -640,7 +646,7 @@ int launch_route_fused(const void* Q, const void* K, int B, int Hq, int Hkv, int
   const size_t kn_bytes = (sizeof(float) * (size_t)B * Hq * Nmax + 255) & ~size_t(255);
   float* scores = reinterpret_cast<float*>(static_cast<char*>(ws) + 256 + kn_bytes);
   const long long hb = heads_per_batch(B, Hq, Nmax);
-  const int smem = (int)(sizeof(float) * (TR * kHeadDim + TK * kKsStride));
+  const int smem = (int)(sizeof(float) * (TR * kHeadDim + 32 * kFusedKC * kKsStride));
   cudaError_t e = cudaFuncSetAttribute(route_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   int dev = 0, sms = 0, per_sm = 0;
   if (e == cudaSuccess) e = cudaGetDevice(&dev);
