@@ -183,8 +183,13 @@ def select_budget(S: np.ndarray, off: np.ndarray, n_chunks: np.ndarray, budget, 
 def budget_near_tie(S_row: np.ndarray, lens: np.ndarray, i: int, budget: int, recent: int, k_max: int,
                     rel: float = 1e-5) -> bool:
     """The kept set can change under a swap of two ranked chunks whose scores
-    differ by less than rel * max_j |S[i, j]| anywhere in the ranked prefix
-    the rule inspects (its taken chunks and the next one)."""
+    differ by less than rel * max_j |S[i, j]| (j over every earlier chunk,
+    window included) anywhere in the ranked prefix the rule inspects.
+
+    The walk takes ranks 0 .. t-1 in order (t = chunks it took) and stops
+    without looking at rank t's identity, so the adjacent pairs that decide
+    the set are (0,1), ..., (t-1,t) -- the taken chunks and the next one.
+    """
     r = min(recent, i, k_max)
     c = i - r
     if c < 2:
@@ -192,12 +197,12 @@ def budget_near_tie(S_row: np.ndarray, lens: np.ndarray, i: int, budget: int, re
     kept = select_budget_row(S_row, lens, i, budget, recent, k_max)
     t = len(kept) - 1 - r                # ranked chunks taken
     last = min(t + 1, c)                 # ranks 0 .. last-1 decide the set
+    if last < 2:
+        return False
     srt = np.sort(S_row[:c])[::-1]
     scale = float(np.max(np.abs(S_row[:i])))
-    gaps = srt[: last - 1] - srt[1:last] if last >= 2 else np.array([])
-    if last < c:                         # the boundary pair
-        gaps = np.append(gaps, srt[last - 1] - srt[last])
-    return bool(gaps.size and gaps.min() < rel * scale)
+    gaps = srt[: last - 1] - srt[1:last]
+    return bool(gaps.min() < rel * scale)
 
 
 # ---------------------------------------------------------------- a4: CSR

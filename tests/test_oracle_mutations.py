@@ -33,6 +33,9 @@ _PINS = [
     (pins.test_budget_uniform_lengths_is_topk_of_budget_over_length, {}),
     (pins.test_budget_zero_keeps_recent_window_only, {}),
     (pins.test_budget_invariants_random, {}),
+    (pins.test_budget_near_tie_hand_cases, {}),
+    (pins.test_density_by_hand, {}),
+    (pins.test_bf16_upcast_bit_patterns, {}),
 ]
 
 
@@ -129,8 +132,84 @@ def _budget_window_uncounted(S_row, lens, i, budget, recent, k_max):
     return _orig["select_budget_row"](S_row, lens, i, budget + extra, recent, k_max)
 
 
+def _near_tie_signed_scale(S_row, lens, i, budget, recent, k_max, rel=1e-5):
+    """Band relative to max S instead of max |S|."""
+    r = min(recent, i, k_max)
+    c = i - r
+    t = len(dhsa.select_budget_row(S_row, lens, i, budget, recent, k_max)) - 1 - r
+    last = min(t + 1, c)
+    if c < 2 or last < 2:
+        return False
+    srt = np.sort(S_row[:c])[::-1]
+    return bool(np.min(srt[: last - 1] - srt[1:last]) < rel * float(np.max(S_row[:i])))
+
+
+def _near_tie_past_boundary(S_row, lens, i, budget, recent, k_max, rel=1e-5):
+    """Also counts the pair just past the boundary (ranks t and t+1)."""
+    if _orig["budget_near_tie"](S_row, lens, i, budget, recent, k_max, rel):
+        return True
+    r = min(recent, i, k_max)
+    c = i - r
+    t = len(dhsa.select_budget_row(S_row, lens, i, budget, recent, k_max)) - 1 - r
+    srt = np.sort(S_row[:c])[::-1]
+    scale = float(np.max(np.abs(S_row[:i])))
+    return bool(t + 1 < c and srt[t] - srt[t + 1] < rel * scale)
+
+
+def _near_tie_no_boundary(S_row, lens, i, budget, recent, k_max, rel=1e-5):
+    """Only gaps between taken chunks; the (last taken, next) pair dropped."""
+    r = min(recent, i, k_max)
+    c = i - r
+    t = len(dhsa.select_budget_row(S_row, lens, i, budget, recent, k_max)) - 1 - r
+    if t < 2:
+        return False
+    srt = np.sort(S_row[:c])[::-1]
+    scale = float(np.max(np.abs(S_row[:i])))
+    return bool(np.min(srt[: t - 1] - srt[1:t]) < rel * scale)
+
+
+def _near_tie_window_ignored(S_row, lens, i, budget, recent, k_max, rel=1e-5):
+    """Ranks taken over every earlier chunk, window chunks included."""
+    return _orig["budget_near_tie"](S_row, lens, i, budget, 0, k_max, rel)
+
+
+def _near_tie_scale_without_window(S_row, lens, i, budget, recent, k_max, rel=1e-5):
+    """Scale from the ranked candidates only (the window's scores left out)."""
+    r = min(recent, i, k_max)
+    s = np.array(S_row, dtype=np.float64)
+    if r > 0:
+        s[i - r:i] = 0.0
+    return _orig["budget_near_tie"](s, lens, i, budget, recent, k_max, rel)
+
+
+def _density_half_square(off, n_chunks, sel, L):
+    """Causal pairs taken as L^2 / 2."""
+    return float(dhsa.kept_pairs(off, n_chunks, sel).mean() / (L * L / 2))
+
+
+def _density_strict_causal(off, n_chunks, sel, L):
+    """Causal pairs taken as L(L-1)/2 (the diagonal left out)."""
+    return float(dhsa.kept_pairs(off, n_chunks, sel).mean() / (L * (L - 1) / 2))
+
+
+def _density_summed(off, n_chunks, sel, L):
+    """Heads summed instead of averaged."""
+    return float(dhsa.kept_pairs(off, n_chunks, sel).sum() / (L * (L + 1) / 2))
+
+
+def _bf16_as_f16(u16):
+    """Bit patterns read as IEEE half precision."""
+    return np.asarray(u16).astype(np.uint16).view(np.float16).astype(np.float64)
+
+
+def _bf16_short_shift(u16):
+    """Shifted by 15 instead of 16."""
+    return (np.asarray(u16).astype(np.uint32) << 15).view(np.float32).astype(np.float64)
+
+
 _orig = {name: getattr(dhsa, name) for name in
-         ("chunk_pool", "chunk_scores", "select_row", "attn_chunk", "select_budget_row")}
+         ("chunk_pool", "chunk_scores", "select_row", "attn_chunk", "select_budget_row", "budget_near_tie",
+          "density", "bf16_to_f64")}
 
 SLIPS = [
     ("chunk_pool", _pool_mean),
@@ -143,6 +222,16 @@ SLIPS = [
     ("attn_chunk", _attn_strict_causal),
     ("select_budget_row", _budget_strict),
     ("select_budget_row", _budget_window_uncounted),
+    ("budget_near_tie", _near_tie_signed_scale),
+    ("budget_near_tie", _near_tie_past_boundary),
+    ("budget_near_tie", _near_tie_no_boundary),
+    ("budget_near_tie", _near_tie_window_ignored),
+    ("budget_near_tie", _near_tie_scale_without_window),
+    ("density", _density_half_square),
+    ("density", _density_strict_causal),
+    ("density", _density_summed),
+    ("bf16_to_f64", _bf16_as_f16),
+    ("bf16_to_f64", _bf16_short_shift),
 ]
 
 

@@ -406,3 +406,36 @@ def test_budget_vector_matches_per_row_scalar():
             for i in range(n):
                 want = dhsa.select_budget_row(S[b, hq, i], lens, i, int(budgets[b, hq, i]), 1, 5)
                 assert sel[b][hq][i].tolist() == want.tolist()
+
+
+def test_budget_near_tie_hand_cases():
+    g = json.load(open(os.path.join(GOLDEN, "budget_near_tie_cases.json")))
+    lens = np.array(g["lens"])
+    for c in g["cases"]:
+        got = dhsa.budget_near_tie(np.array(c["S"]), lens, g["i"], c["budget"], c["recent"], c["k_max"])
+        assert got == c["expect"], c["name"]
+
+
+# ------------------------------------------------------------ density, bf16 upcast
+def test_density_by_hand():
+    # the 6-token layout of test_kept_pairs_by_hand: causal pairs 6*7/2 = 21
+    off = np.array([[0, 2, 5, 6]], dtype=np.int32)
+    nc = np.array([3], dtype=np.int32)
+    sel_a = [np.array([0]), np.array([0, 1]), np.array([1, 2])]        # 19 kept pairs
+    sel_b = [np.array([0]), np.array([1]), np.array([2])]              # 3 + 6 + 1 = 10
+    assert dhsa.density(off, nc, [[sel_a]], 6) == 19 / 21
+    # two heads average: (19 + 10) / 2 over 21
+    assert dhsa.density(off, nc, [[sel_a, sel_b]], 6) == 14.5 / 21
+
+
+def test_bf16_upcast_bit_patterns():
+    bits = np.array([0x3F80, 0xC020, 0x0001, 0xFF80, 0x7F80, 0x8000, 0x4049, 0x7F7F, 0x0080, 0x3F81],
+                    dtype=np.uint16)
+    want = [1.0, -2.5, 2.0 ** -133, -math.inf, math.inf, -0.0, 3.140625, (2 - 2 ** -7) * 2.0 ** 127,
+            2.0 ** -126, 1 + 2 ** -7]
+    got = dhsa.bf16_to_f64(bits)
+    assert got.dtype == np.float64
+    assert got.tolist() == want
+    assert math.copysign(1.0, got[5]) == -1.0             # the sign of -0 survives
+    # a quiet NaN pattern stays NaN
+    assert math.isnan(dhsa.bf16_to_f64(np.array([0x7FC0], dtype=np.uint16))[0])
