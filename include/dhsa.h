@@ -55,8 +55,11 @@ typedef enum {
 } dhsa_status_t;
 
 /* Device status word bits, as returned in *device_flags by dhsa_check_device_status. */
-#define DHSA_DEVFLAG_WAIT_TIMEOUT 0x1  /* a pipeline wait in the attention kernel gave up */
-#define DHSA_DEVFLAG_BAD_OFFSETS 0x2   /* dhsa_validate_offsets found a bad offsets table */
+#define DHSA_DEVFLAG_WAIT_TIMEOUT 0x1  /* a pipeline wait of the attention kernels or a grid barrier of
+                                          the fused routing gave up (that launch's results are undefined) */
+#define DHSA_DEVFLAG_BAD_OFFSETS 0x2   /* an inconsistent offsets table: found by dhsa_validate_offsets,
+                                          or met (and clamped) by pooling, or met by the attention's
+                                          work-list builder (the batch element is then skipped) */
 #define DHSA_DEVFLAG_BAD_SELECTION 0x4 /* the CSR builder met a selected chunk outside [0, i] */
 
 /* Human-readable name of a status code (static string, never NULL). */
@@ -92,6 +95,9 @@ int dhsa_validate_offsets(const int32_t* off, const int32_t* n_chunks, int B, in
  *    X   bf16  [B, H, L, head_dim]  (call once with Q, H = Hq; once with K, H = Hkv)
  *    Xp  fp32  [B, H, Nmax, head_dim], written in full: rows c >= n_chunks[b]
  *        are set to zero. Sums are accumulated in fp32.
+ *    A chunk count outside [0, Nmax] or a chunk bound outside [0, L] is
+ *    clamped before any row is read and sets DHSA_DEVFLAG_BAD_OFFSETS; no
+ *    read leaves the head's L rows.
  * ------------------------------------------------------------------------- */
 int dhsa_chunk_pool(const void* X, int B, int H, int L, int head_dim, const int32_t* off,
                     const int32_t* n_chunks, int Nmax, float* Xp, void* stream);
@@ -175,13 +181,15 @@ int dhsa_chunk_score_select_budget(const float* Qp, const float* Kp, int B, int 
  *    Does what dhsa_chunk_pool_qk followed by dhsa_chunk_score_topk do, with
  *    the same results bit for bit, as one cooperative launch: pooling of Q
  *    and K, key norms and score tiles, then the selection, separated by
- *    grid-wide barriers (each bounded: a barrier that waits more than 1 s
- *    sets DHSA_DEVFLAG_WAIT_TIMEOUT). Arguments and layouts are those of the
- *    two calls; Qp and Kp are written as by 1b.
+ *    grid-wide barriers (each bounded: a block that waits more than 1 s at a
+ *    barrier sets DHSA_DEVFLAG_WAIT_TIMEOUT and an abort word, and every
+ *    block then leaves the kernel; the outputs of that launch are undefined).
+ *    Arguments and layouts are those of the two calls; Qp and Kp are written
+ *    as by 1b.
  *    workspace: dhsa_route_fused_workspace_size(B, Hq, Nmax) bytes (equal to
- *    dhsa_score_topk_workspace_size; its first 4 bytes hold the barrier
- *    count, reset by this call on `stream`). Calls sharing a workspace must
- *    not overlap on the GPU.
+ *    dhsa_score_topk_workspace_size; its first 8 bytes hold the barrier
+ *    count and the abort word, reset by this call on `stream`). Calls
+ *    sharing a workspace must not overlap on the GPU.
  * ------------------------------------------------------------------------- */
 size_t dhsa_route_fused_workspace_size(int B, int Hq, int Nmax);
 int dhsa_route_fused(const void* Q, const void* K, int B, int Hq, int Hkv, int L, int head_dim, const int32_t* off,
@@ -223,7 +231,10 @@ int dhsa_build_block_csr(const int32_t* sel, const int32_t* n_sel, int B, int Hq
  *    masked key contributes 0 * V[s]).
  *
  *    row_ptr / col_idx as written by 3. (cost may be NULL; it is not read yet).
- *    O bf16 [B, Hq, L, 128]; every token row of every head is written.
+ *    A col_idx entry outside [0, i] is clamped into it (3. flags such rows).
+ *    O bf16 [B, Hq, L, 128]; every token row of every head is written, except
+ *    in a batch element whose offsets table is inconsistent (that element is
+ *    skipped and DHSA_DEVFLAG_BAD_OFFSETS set).
  *    workspace: dhsa_sparse_attn_workspace_size(B, Hq, L, Nmax) bytes.
  * ------------------------------------------------------------------------- */
 size_t dhsa_sparse_attn_workspace_size(int B, int Hq, int L, int Nmax);
@@ -290,6 +301,27 @@ int dhsa_sparse_attn_fwd_tiles(const void* Q, const void* K, const void* V, int 
                                int head_dim, const int32_t* off, const int32_t* n_chunks, int Nmax,
                                const int32_t* row_ptr, const int32_t* col_idx, float softmax_scale, int short_tiles,
                                void* O, void* workspace, size_t workspace_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * 5. Test hook of the bounded device waits.
+ *    The paper has no counterpart. Every wait of the pipelined kernels gives
+ *    up after 1 s and reports DHSA_DEVFLAG_WAIT_TIMEOUT instead of hanging;
+ *    this hook lets a test make such a wait run out on purpose, without any
+ *    fault, so that the path is exercised:
+ *      mode 1: the next attention launch (4., 4b. or 4c. with 128-row tiles)
+ *              holds back its scheduler, so the other roles' first wait --
+ *              which precedes every copy and MMA -- runs out after limit_ns;
+ *              the CTAs record the flag, free their TMEM and return without
+ *              writing O.
+ *      mode 2: the next dhsa_route_fused launch has block 0 arrive late at
+ *              its first grid barrier; the other blocks give up after
+ *              limit_ns, set the abort word, and all blocks leave.
+ *      mode 0: disarm.
+ *    The hook is one-shot (the launch that uses it disarms it) and host-side
+ *    state of the library: not thread-safe, for tests only.
+ *    limit_ns: 1 .. 100,000,000 for modes 1 and 2 (DHSA_ERR_INVALID_ARG else).
+ * ------------------------------------------------------------------------- */
+int dhsa_debug_arm_wait_timeout(int mode, uint64_t limit_ns);
 
 #ifdef __cplusplus
 }

@@ -62,6 +62,7 @@ _SIGNATURES = {
     "dhsa_sparse_attn_tiles_workspace_size": (_SZ, [_I, _I, _I, _I, _I]),
     "dhsa_sparse_attn_fwd_tiles": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _I, _P, _P, _F, _I, _P, _P, _SZ,
                                         _P]),
+    "dhsa_debug_arm_wait_timeout": (_I, [_I, _c.c_uint64]),
 }
 
 _lib: Optional[ctypes.CDLL] = None
@@ -123,6 +124,13 @@ def check_device_status() -> int:
         raise DHSAError(st, "dhsa_check_device_status", load().dhsa_last_cuda_error() if st == 3 else 0,
                         flags.value)
     return flags.value
+
+
+def debug_arm_wait_timeout(mode: int, limit_ns: int = 0):
+    """Test hook of the bounded device waits (include/dhsa.h, 5): mode 1 makes
+    the next attention launch's first waits run out after limit_ns, mode 2
+    the next fused-routing launch's first grid barrier; 0 disarms."""
+    _check(load().dhsa_debug_arm_wait_timeout(mode, limit_ns), "dhsa_debug_arm_wait_timeout")
 
 
 def validate_offsets(off: torch.Tensor, n_chunks: torch.Tensor, L: int):

@@ -7,9 +7,10 @@
 namespace dhsa {
 
 int launch_chunk_pool(const void* X, int B, int H, int L, const int32_t* off, const int32_t* n_chunks, int Nmax,
-                      float* Xp, cudaStream_t stream);
+                      float* Xp, unsigned int* status, cudaStream_t stream);
 int launch_chunk_pool_qk(const void* Q, const void* K, int B, int Hq, int Hkv, int L, const int32_t* off,
-                         const int32_t* n_chunks, int Nmax, float* Qp, float* Kp, cudaStream_t stream);
+                         const int32_t* n_chunks, int Nmax, float* Qp, float* Kp, unsigned int* status,
+                         cudaStream_t stream);
 int launch_validate_offsets(const int32_t* off, const int32_t* n_chunks, int B, int Nmax, int L,
                             unsigned int* status, cudaStream_t stream);
 int score_topk_stride(int k, int Nmax);
@@ -18,7 +19,8 @@ int launch_score_topk(const float* Qp, const float* Kp, int B, int Hq, int Hkv, 
                       int k, int32_t* sel, int32_t* n_sel, void* ws, cudaStream_t stream);
 int launch_route_fused(const void* Q, const void* K, int B, int Hq, int Hkv, int L, const int32_t* off,
                        const int32_t* n_chunks, int Nmax, int k, float* Qp, float* Kp, int32_t* sel, int32_t* n_sel,
-                       void* ws, unsigned int* status, cudaStream_t stream);
+                       void* ws, unsigned int* status, unsigned long long limit_ns, unsigned long long hold_ns,
+                       cudaStream_t stream);
 int score_budget_max_chunks();
 int launch_score_budget(const float* Qp, const float* Kp, int B, int Hq, int Hkv, int Nmax, const int32_t* off,
                         const int32_t* n_chunks, int budget, const int32_t* budgets, int recent, int k_max,
@@ -45,6 +47,19 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 }  // namespace
 
 void set_last_cuda_error(cudaError_t e) { t_last_cuda_error = (int)e; }
+
+namespace {
+// armed test hook of the bounded waits (dhsa_debug_arm_wait_timeout)
+int g_wait_test_mode = 0;
+unsigned long long g_wait_test_limit_ns = 0;
+}  // namespace
+
+bool take_wait_test(int mode, unsigned long long* limit_ns) {
+  if (g_wait_test_mode != mode) return false;
+  *limit_ns = g_wait_test_limit_ns;
+  g_wait_test_mode = 0;
+  return true;
+}
 
 unsigned int* device_status_ptr() {
   int dev = 0;
@@ -109,7 +124,7 @@ const char* dhsa_status_string(int status) {
 
 int dhsa_last_cuda_error(void) { return t_last_cuda_error; }
 
-int dhsa_version(void) { return 200; }   // 0.2.0: pooling of Q and K in one call, budget selection, query-tile policy
+int dhsa_version(void) { return 300; }   // 0.3.0: wait-timeout test hook; offsets clamped by pooling and the work list
 
 int dhsa_check_device_status(void* stream, uint32_t* device_flags) {
   if (device_flags) *device_flags = 0;
@@ -143,7 +158,9 @@ int dhsa_chunk_pool(const void* X, int B, int H, int L, int head_dim, const int3
   if (!X || !Xp || !aligned16(X) || !aligned16(Xp)) return DHSA_ERR_INVALID_ARG;
   if (head_dim != kHeadDim) return DHSA_ERR_UNSUPPORTED;
   if ((st = check_device_sm100()) != DHSA_OK) return st;
-  return launch_chunk_pool(X, B, H, L, off, n_chunks, Nmax, Xp, static_cast<cudaStream_t>(stream));
+  unsigned int* status = device_status_ptr();
+  if (!status) return DHSA_ERR_CUDA;
+  return launch_chunk_pool(X, B, H, L, off, n_chunks, Nmax, Xp, status, static_cast<cudaStream_t>(stream));
 }
 
 int dhsa_chunk_pool_qk(const void* Q, const void* K, int B, int Hq, int Hkv, int L, int head_dim,
@@ -155,7 +172,10 @@ int dhsa_chunk_pool_qk(const void* Q, const void* K, int B, int Hq, int Hkv, int
     return DHSA_ERR_INVALID_ARG;
   if (head_dim != kHeadDim) return DHSA_ERR_UNSUPPORTED;
   if ((st = check_device_sm100()) != DHSA_OK) return st;
-  return launch_chunk_pool_qk(Q, K, B, Hq, Hkv, L, off, n_chunks, Nmax, Qp, Kp, static_cast<cudaStream_t>(stream));
+  unsigned int* status = device_status_ptr();
+  if (!status) return DHSA_ERR_CUDA;
+  return launch_chunk_pool_qk(Q, K, B, Hq, Hkv, L, off, n_chunks, Nmax, Qp, Kp, status,
+                              static_cast<cudaStream_t>(stream));
 }
 
 int dhsa_sel_stride(int k, int Nmax) {
@@ -201,8 +221,13 @@ int dhsa_route_fused(const void* Q, const void* K, int B, int Hq, int Hkv, int L
   if ((st = check_device_sm100()) != DHSA_OK) return st;
   unsigned int* status = device_status_ptr();
   if (!status) return DHSA_ERR_CUDA;
+  unsigned long long limit_ns = kWaitLimitNs, hold_ns = 0, test_ns = 0;
+  if (take_wait_test(2, &test_ns)) {   // block 0 arrives late; the others give up after test_ns
+    limit_ns = test_ns;
+    hold_ns = 4 * test_ns + 1000000ull;
+  }
   return launch_route_fused(Q, K, B, Hq, Hkv, L, off, n_chunks, Nmax, k, Qp, Kp, sel, n_sel, workspace, status,
-                            static_cast<cudaStream_t>(stream));
+                            limit_ns, hold_ns, static_cast<cudaStream_t>(stream));
 }
 
 int dhsa_budget_max_chunks(void) { return score_budget_max_chunks(); }
@@ -300,6 +325,14 @@ int dhsa_sparse_attn_fwd_noalloc(const void* Q, const void* K, const void* V, in
   if ((st = noalloc_scratch_ptr(&scratch)) != DHSA_OK) return st;
   return launch_sparse_attn(Q, K, V, B, Hq, Hkv, L, off, n_chunks, Nmax, row_ptr, col_idx, softmax_scale, 0, O,
                             scratch, status, static_cast<cudaStream_t>(stream));
+}
+
+int dhsa_debug_arm_wait_timeout(int mode, uint64_t limit_ns) {
+  if (mode < 0 || mode > 2) return DHSA_ERR_INVALID_ARG;
+  if (mode != 0 && (limit_ns == 0 || limit_ns > 100000000ull)) return DHSA_ERR_INVALID_ARG;
+  g_wait_test_mode = mode;
+  g_wait_test_limit_ns = limit_ns;
+  return DHSA_OK;
 }
 
 }  // extern "C"

@@ -11,8 +11,8 @@ namespace dhsa {
 
 long long attn_cap_long(int B, int Hq, int L, int Nmax, int policy);
 long long attn_cap_short(int B, int Hq, int L, int Nmax, int policy);
-int launch_build_items(const int32_t* off, const int32_t* n_chunks, int B, int Hq, int G, int Nmax, int policy,
-                       const AttnWork& w, cudaStream_t stream);
+int launch_build_items(const int32_t* off, const int32_t* n_chunks, int B, int Hq, int G, int L, int Nmax,
+                       int policy, const AttnWork& w, unsigned int* status, cudaStream_t stream);
 int launch_sparse_attn_long(const AttnWork& w, const void* Q, const void* K, const void* V, int B, int Hq, int Hkv,
                             int L, const int32_t* off, int Nmax, const int32_t* row_ptr, const int32_t* col_idx,
                             float softmax_scale, void* O, unsigned int* status, cudaStream_t stream);
@@ -40,7 +40,7 @@ int launch_sparse_attn(const void* Q, const void* K, const void* V, int B, int H
   w.counter_short = head + 3;
   w.items_long = reinterpret_cast<int4*>(static_cast<char*>(ws) + 256);
   w.items_short = w.items_long + w.cap_long;
-  int st = launch_build_items(off, n_chunks, B, Hq, Hq / Hkv, Nmax, policy, w, stream);
+  int st = launch_build_items(off, n_chunks, B, Hq, Hq / Hkv, L, Nmax, policy, w, status, stream);
   if (st == DHSA_OK)
     st = launch_sparse_attn_long(w, Q, K, V, B, Hq, Hkv, L, off, Nmax, row_ptr, col_idx, softmax_scale, O, status,
                                  stream);

@@ -64,7 +64,6 @@ constexpr uint32_t kQTile = 2 * kQHalf;
 constexpr uint32_t kPTile = BN * NQ * 2;        // P^T: 128 key rows x 64 bf16
 constexpr uint32_t kTmemCols = 256;
 constexpr uint32_t kTmemO = 192;                // O^T columns
-constexpr uint64_t kWaitLimitNs = 1000000000ull;
 constexpr float kRaise = 32.0f;                 // log2 headroom before a column max must rise
 
 struct ShortMaps {

@@ -29,6 +29,14 @@ inline int cuda_status(cudaError_t e) {
   return DHSA_ERR_CUDA;
 }
 
+// Wall-clock limit of every bounded device wait (1 s).
+constexpr unsigned long long kWaitLimitNs = 1000000000ull;
+
+// Test hook of the bounded waits: true (once) when dhsa_debug_arm_wait_timeout
+// armed `mode` (1 = attention, 2 = fused routing); *limit_ns gets the short
+// limit the launch must use. Host side, not thread-safe.
+bool take_wait_test(int mode, unsigned long long* limit_ns);
+
 // Launch check: picks up configuration errors of the launch just made.
 inline int launch_status() { return cuda_status(cudaGetLastError()); }
 

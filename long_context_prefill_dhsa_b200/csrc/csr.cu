@@ -20,8 +20,15 @@ namespace {
 
 constexpr int kScanThreads = 1024;
 
+// A count outside [0, stride] (a malformed selection) is clamped into it
+// here and in fill_rows_kernel alike, so the CSR never outgrows
+// dhsa_csr_nnz_upper; fill_rows_kernel flags the row.
+__device__ __forceinline__ int row_count(const int32_t* n_sel, long long r, int stride) {
+  return min(max(n_sel[r], 0), stride);
+}
+
 __global__ void __launch_bounds__(kScanThreads) scan_rows_kernel(const int32_t* __restrict__ n_sel, long long R,
-                                                                 int32_t* __restrict__ row_ptr) {
+                                                                 int stride, int32_t* __restrict__ row_ptr) {
   // exclusive scan in blocks of 4 * kScanThreads rows: each thread reads four
   // consecutive counts (coalesced across the block), scans them, and the
   // block scans the thread totals; a running carry links the blocks
@@ -35,7 +42,7 @@ __global__ void __launch_bounds__(kScanThreads) scan_rows_kernel(const int32_t* 
     const long long r0 = base + 4LL * t;
     int v[4];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) v[q] = (r0 + q < R) ? n_sel[r0 + q] : 0;
+    for (int q = 0; q < 4; ++q) v[q] = (r0 + q < R) ? row_count(n_sel, r0 + q, stride) : 0;
     const long long local = (long long)v[0] + v[1] + v[2] + v[3];
     long long incl = local;
 #pragma unroll
@@ -83,18 +90,19 @@ __global__ void __launch_bounds__(256) fill_rows_kernel(const int32_t* __restric
   const int i = (int)(r % Nmax);
   const int b = (int)(r / ((long long)Hq * Nmax));
   const int32_t* ob = off + (long long)b * (Nmax + 1);
-  const int cnt = n_sel[r];
+  const int cnt = row_count(n_sel, r, stride);
   const int32_t* src = sel + r * stride;
   int32_t* dst = col_idx + row_ptr[r];
-  const int n = n_chunks[b];
+  const int n = min(max(n_chunks[b], 0), Nmax);   // a count outside [0, Nmax] is clamped
   long long keys = 0;
-  bool bad = false;
+  bool bad = cnt != n_sel[r];
   for (int q = lane; q < cnt; q += 32) {
     const int j = src[q];
-    dst[q] = j;
     if (j < 0 || j > i || i >= n) {
       bad = true;
+      dst[q] = min(max(j, 0), i);   // stored in range, flagged
     } else {
+      dst[q] = j;
       keys += ob[j + 1] - ob[j];
     }
   }
@@ -112,7 +120,7 @@ int launch_build_csr(const int32_t* sel, const int32_t* n_sel, int B, int Hq, in
                      const int32_t* n_chunks, int32_t* row_ptr, int32_t* col_idx, int64_t* cost,
                      unsigned int* status, cudaStream_t stream) {
   const long long R = (long long)B * Hq * Nmax;
-  scan_rows_kernel<<<1, kScanThreads, 0, stream>>>(n_sel, R, row_ptr);
+  scan_rows_kernel<<<1, kScanThreads, 0, stream>>>(n_sel, R, score_topk_stride(k, Nmax), row_ptr);
   int st = launch_status();
   if (st != DHSA_OK) return st;
   const int threads = 256;

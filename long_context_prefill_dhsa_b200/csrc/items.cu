@@ -26,6 +26,15 @@ __device__ __forceinline__ int2 tile_counts(int len, int policy) {
   return tail <= kShortRows ? make_int2(nt - 1, 1) : make_int2(nt, 0);
 }
 
+// A batch element's offsets table is consistent when 1 <= n <= Nmax,
+// off[0] = 0, off[n] = L and every chunk is non-empty. An inconsistent one
+// contributes no items (its tile counts could overrun the lists) and sets
+// DHSA_DEVFLAG_BAD_OFFSETS.
+__device__ __forceinline__ bool chunk_ok(const int32_t* ob, int c, int n, int L) {
+  const int s = ob[c], e = ob[c + 1];
+  return s >= 0 && e > s && e <= L && (c > 0 || s == 0) && (c < n - 1 || e == L);
+}
+
 // Both lists are ordered (b, kv head, chunk, query head within the group,
 // tile), so CTAs running at the same time share the K/V of one kv head in L2.
 // One CTA per (query head, batch element) writes that head's items; it
@@ -33,14 +42,23 @@ __device__ __forceinline__ int2 tile_counts(int len, int policy) {
 // totals of the earlier ones for its base offsets).
 __global__ void __launch_bounds__(1024) build_items_kernel(const int32_t* __restrict__ off,
                                                            const int32_t* __restrict__ n_chunks, int B, int Hq,
-                                                           int G, int Nmax, int policy, AttnWork w) {
+                                                           int G, int L, int Nmax, int policy, AttnWork w,
+                                                           unsigned int* status) {
   __shared__ int2 warp_sum[32];
   __shared__ int2 carry_s;
   const int t = threadIdx.x, lane = t & 31, wp = t >> 5;
   const int hq = blockIdx.x, b = blockIdx.y;
   const int hkv = hq / G, gq = hq % G;
-  auto totals_of = [&](int bb) -> int2 {   // (long, short) tiles of batch element bb
+  auto valid = [&](int bb) -> bool {
     const int n = n_chunks[bb];
+    const int32_t* ob = off + (long long)bb * (Nmax + 1);
+    bool bad = n < 1 || n > Nmax;
+    if (!bad)
+      for (int c = t; c < n; c += 1024) bad = bad || !chunk_ok(ob, c, n, L);
+    return !__syncthreads_or(bad);
+  };
+  auto totals_of = [&](int bb) -> int2 {   // (long, short) tiles of batch element bb (0 if inconsistent)
+    const int n = valid(bb) ? n_chunks[bb] : 0;
     const int32_t* ob = off + (long long)bb * (Nmax + 1);
     int2 local = make_int2(0, 0);
     for (int c = t; c < n; c += 1024) {
@@ -70,7 +88,9 @@ __global__ void __launch_bounds__(1024) build_items_kernel(const int32_t* __rest
     base_s += (long long)Hq * tb.y;
   }
   const int2 Tb = totals_of(b);
-  const int n = n_chunks[b];
+  const bool ok_b = valid(b);
+  if (!ok_b && hq == 0 && t == 0) raise_device_flag(status, DHSA_DEVFLAG_BAD_OFFSETS);
+  const int n = ok_b ? n_chunks[b] : 0;
   const int32_t* ob = off + (long long)b * (Nmax + 1);
   __syncthreads();
   if (t == 0) carry_s = make_int2(0, 0);
@@ -132,9 +152,9 @@ long long attn_cap_short(int B, int Hq, int L, int Nmax, int policy) {
   return (long long)B * Hq * ((long long)Nmax + ceil_div(L, kShortRows));
 }
 
-int launch_build_items(const int32_t* off, const int32_t* n_chunks, int B, int Hq, int G, int Nmax, int policy,
-                       const AttnWork& w, cudaStream_t stream) {
-  build_items_kernel<<<dim3(Hq, B), 1024, 0, stream>>>(off, n_chunks, B, Hq, G, Nmax, policy, w);
+int launch_build_items(const int32_t* off, const int32_t* n_chunks, int B, int Hq, int G, int L, int Nmax,
+                       int policy, const AttnWork& w, unsigned int* status, cudaStream_t stream) {
+  build_items_kernel<<<dim3(Hq, B), 1024, 0, stream>>>(off, n_chunks, B, Hq, G, L, Nmax, policy, w, status);
   return launch_status();
 }
 

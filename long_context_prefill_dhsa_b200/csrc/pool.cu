@@ -21,9 +21,10 @@ namespace {
 __global__ void __launch_bounds__(256) chunk_pool_kernel(const uint4* __restrict__ X, int H, int L,
                                                          const int32_t* __restrict__ off,
                                                          const int32_t* __restrict__ n_chunks, int Nmax,
-                                                         long long n_rows, float* __restrict__ Xp) {
+                                                         long long n_rows, float* __restrict__ Xp,
+                                                         unsigned int* status) {
   const long long warp = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  if (warp < n_rows) pool_row(X, H, L, off, n_chunks, Nmax, warp, Xp);
+  if (warp < n_rows) pool_row(X, H, L, off, n_chunks, Nmax, warp, Xp, status);
 }
 
 // Q and K in one launch: warps [0, rows_q) pool Q, the rest pool K, so the
@@ -32,10 +33,11 @@ __global__ void __launch_bounds__(256) chunk_pool_qk_kernel(const uint4* __restr
                                                             int Hq, int Hkv, int L, const int32_t* __restrict__ off,
                                                             const int32_t* __restrict__ n_chunks, int Nmax,
                                                             long long rows_q, long long rows_k,
-                                                            float* __restrict__ Qp, float* __restrict__ Kp) {
+                                                            float* __restrict__ Qp, float* __restrict__ Kp,
+                                                            unsigned int* status) {
   const long long warp = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  if (warp < rows_q) pool_row(Q, Hq, L, off, n_chunks, Nmax, warp, Qp);
-  else if (warp < rows_q + rows_k) pool_row(K, Hkv, L, off, n_chunks, Nmax, warp - rows_q, Kp);
+  if (warp < rows_q) pool_row(Q, Hq, L, off, n_chunks, Nmax, warp, Qp, status);
+  else if (warp < rows_q + rows_k) pool_row(K, Hkv, L, off, n_chunks, Nmax, warp - rows_q, Kp, status);
 }
 
 __global__ void validate_offsets_kernel(const int32_t* __restrict__ off, const int32_t* __restrict__ n_chunks,
@@ -59,23 +61,24 @@ __global__ void validate_offsets_kernel(const int32_t* __restrict__ off, const i
 }  // namespace
 
 int launch_chunk_pool(const void* X, int B, int H, int L, const int32_t* off, const int32_t* n_chunks, int Nmax,
-                      float* Xp, cudaStream_t stream) {
+                      float* Xp, unsigned int* status, cudaStream_t stream) {
   const long long n_rows = (long long)B * H * Nmax;
   const int threads = 256;
   const long long blocks = (n_rows * 32 + threads - 1) / threads;
   chunk_pool_kernel<<<(unsigned)blocks, threads, 0, stream>>>(static_cast<const uint4*>(X), H, L, off, n_chunks,
-                                                               Nmax, n_rows, Xp);
+                                                               Nmax, n_rows, Xp, status);
   return launch_status();
 }
 
 int launch_chunk_pool_qk(const void* Q, const void* K, int B, int Hq, int Hkv, int L, const int32_t* off,
-                         const int32_t* n_chunks, int Nmax, float* Qp, float* Kp, cudaStream_t stream) {
+                         const int32_t* n_chunks, int Nmax, float* Qp, float* Kp, unsigned int* status,
+                         cudaStream_t stream) {
   const long long rows_q = (long long)B * Hq * Nmax, rows_k = (long long)B * Hkv * Nmax;
   const int threads = 256;
   const long long blocks = ((rows_q + rows_k) * 32 + threads - 1) / threads;
   chunk_pool_qk_kernel<<<(unsigned)blocks, threads, 0, stream>>>(static_cast<const uint4*>(Q),
                                                                   static_cast<const uint4*>(K), Hq, Hkv, L, off,
-                                                                  n_chunks, Nmax, rows_q, rows_k, Qp, Kp);
+                                                                  n_chunks, Nmax, rows_q, rows_k, Qp, Kp, status);
   return launch_status();
 }
 

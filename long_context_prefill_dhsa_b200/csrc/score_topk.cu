@@ -51,11 +51,28 @@ __device__ __forceinline__ unsigned lanemask_lt() {
 
 __host__ __device__ __forceinline__ long long tri(long long i) { return i * (i - 1) / 2; }
 
+// Loads of the pooled vectors, key norms and scores. The separate kernels read
+// buffers an earlier launch wrote and use plain loads; the fused routing
+// kernel reads buffers other blocks of the same launch wrote (after a grid
+// barrier), so its instantiation (kCoh) loads through L2 (ld.global.cg),
+// never through a possibly stale or non-coherent L1 line.
+template <bool kCoh>
+__device__ __forceinline__ float ldf(const float* p) {
+  if constexpr (kCoh) return __ldcg(p);
+  else return *p;
+}
+template <bool kCoh>
+__device__ __forceinline__ float4 ldf4(const float* p) {
+  if constexpr (kCoh) return __ldcg(reinterpret_cast<const float4*>(p));
+  else return *reinterpret_cast<const float4*>(p);
+}
+
 // ------------------------------------------------------------------ 1. key norms
 // one warp: the norm of pooled key row r
+template <bool kCoh>
 __device__ __forceinline__ void key_norm_row(const float* __restrict__ Kp, long long r, float* __restrict__ kn) {
   const int lane = threadIdx.x & 31;
-  const float4 v = reinterpret_cast<const float4*>(Kp + r * kHeadDim)[lane];
+  const float4 v = ldf4<kCoh>(Kp + r * kHeadDim + 4 * lane);
   double s = (double)v.x * v.x + (double)v.y * v.y + (double)v.z * v.z + (double)v.w * v.w;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
@@ -65,7 +82,7 @@ __device__ __forceinline__ void key_norm_row(const float* __restrict__ Kp, long 
 __global__ void __launch_bounds__(256) key_norm_kernel(const float* __restrict__ Kp, long long rows,
                                                        float* __restrict__ kn) {
   const long long r = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  if (r < rows) key_norm_row(Kp, r, kn);
+  if (r < rows) key_norm_row<false>(Kp, r, kn);
 }
 
 // ------------------------------------------------------------------ 2. fp32 score tiles
@@ -73,7 +90,7 @@ __global__ void __launch_bounds__(256) key_norm_kernel(const float* __restrict__
 // rows of ws; a tile is TR query rows x 32 * KC keys (sm: TR * 128 +
 // 32 * KC * 132 floats of shared memory). Every score is one thread's fp32
 // dot product in a fixed order, whatever KC.
-template <int KC>
+template <int KC, bool kCoh>
 __device__ __forceinline__ void score_tile_body(const float* __restrict__ Qp, const float* __restrict__ Kp, int Hq,
                                                 int G, int Nmax, const int32_t* __restrict__ n_chunks, long long bh0,
                                                 int bhl, int rb, int kb, float* __restrict__ ws, float* sm) {
@@ -81,7 +98,7 @@ __device__ __forceinline__ void score_tile_body(const float* __restrict__ Qp, co
   float* Ks = sm + TR * kHeadDim;        // [32 * KC][132]
   const long long bh = bh0 + bhl;
   const int b = (int)(bh / Hq), hq = (int)(bh % Hq);
-  const int n = n_chunks[b];
+  const int n = min(max(n_chunks[b], 0), Nmax);   // a count outside [0, Nmax] is clamped
   const int i0 = rb * TR, j0 = kb * 32 * KC;
   const int i_hi = min(i0 + TR, n);                 // rows [i0, i_hi)
   if (i0 >= n || j0 >= i_hi - 1) return;            // no j < i in this tile
@@ -90,14 +107,14 @@ __device__ __forceinline__ void score_tile_body(const float* __restrict__ Qp, co
     const int r = idx >> 5, c4 = idx & 31;
     const int i = i0 + r;
     float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (i < n) v = reinterpret_cast<const float4*>(Qp + (bh * Nmax + i) * kHeadDim)[c4];
+    if (i < n) v = ldf4<kCoh>(Qp + (bh * Nmax + i) * kHeadDim + 4 * c4);
     reinterpret_cast<float4*>(Qs + r * kHeadDim)[c4] = v;
   }
   for (int idx = threadIdx.x; idx < 32 * KC * 32; idx += blockDim.x) {
     const int r = idx >> 5, c4 = idx & 31;
     const int j = j0 + r;
     float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (j < n) v = reinterpret_cast<const float4*>(Kp + (kv_row0 + j) * kHeadDim)[c4];
+    if (j < n) v = ldf4<kCoh>(Kp + (kv_row0 + j) * kHeadDim + 4 * c4);
     reinterpret_cast<float4*>(Ks + r * kKsStride)[c4] = v;
   }
   __syncthreads();
@@ -142,16 +159,17 @@ __global__ void __launch_bounds__(256, 2) score_tile_kernel(const float* __restr
                                                          const int32_t* __restrict__ n_chunks, long long bh0,
                                                          int n_rb, int n_kb, float* __restrict__ ws) {
   extern __shared__ __align__(16) float sm[];
-  score_tile_body<TK / 32>(Qp, Kp, Hq, G, Nmax, n_chunks, bh0, blockIdx.y, blockIdx.x / n_kb, blockIdx.x % n_kb, ws,
+  score_tile_body<TK / 32, false>(Qp, Kp, Hq, G, Nmax, n_chunks, bh0, blockIdx.y, blockIdx.x / n_kb, blockIdx.x % n_kb, ws,
                           sm);
 }
 
 // ------------------------------------------------------------------ 3. selection
+template <bool kCoh>
 __device__ double exact_score(const float* __restrict__ q, const float* __restrict__ k) {
   double a0 = 0.0, a1 = 0.0, a2 = 0.0, a3 = 0.0;
   for (int d = 0; d < kHeadDim; d += 4) {
-    const float4 x = *reinterpret_cast<const float4*>(q + d);
-    const float4 y = *reinterpret_cast<const float4*>(k + d);
+    const float4 x = ldf4<kCoh>(q + d);
+    const float4 y = ldf4<kCoh>(k + d);
     a0 = fma((double)x.x, (double)y.x, a0);
     a1 = fma((double)x.y, (double)y.y, a1);
     a2 = fma((double)x.z, (double)y.z, a2);
@@ -175,6 +193,7 @@ struct Cut {
   bool all_band;
 };
 
+template <bool kCoh>
 __device__ Cut topm_cut(const float* __restrict__ row, int c, int m, int* hist, const float* __restrict__ qrow,
                         const float* __restrict__ Kp, long long kv_row0, const float* __restrict__ kn) {
   const int lane = threadIdx.x & 31;
@@ -186,7 +205,7 @@ __device__ Cut topm_cut(const float* __restrict__ row, int c, int m, int* hist, 
     for (int q = lane; q < 256; q += 32) hist[q] = 0;
     __syncwarp();
     for (int j = lane; j < c; j += 32) {
-      const unsigned kk = order_key32(row[j]);
+      const unsigned kk = order_key32(ldf<kCoh>(row + j));
       if ((kk & mask) == prefix) atomicAdd(&hist[(kk >> shift) & 255], 1);
     }
     __syncwarp();
@@ -228,10 +247,10 @@ __device__ Cut topm_cut(const float* __restrict__ row, int c, int m, int* hist, 
   const unsigned tu = (prefix & 0x80000000u) ? (prefix & 0x7fffffffu) : ~prefix;
   const double T = (double)__uint_as_float(tu);
   // --- rounding band
-  const float4 qv = reinterpret_cast<const float4*>(qrow)[lane];
+  const float4 qv = ldf4<kCoh>(qrow + 4 * lane);
   double qq = (double)qv.x * qv.x + (double)qv.y * qv.y + (double)qv.z * qv.z + (double)qv.w * qv.w;
   float kmax = 0.f;
-  for (int j = lane; j < c; j += 32) kmax = fmaxf(kmax, kn[kv_row0 + j]);
+  for (int j = lane; j < c; j += 32) kmax = fmaxf(kmax, ldf<kCoh>(kn + kv_row0 + j));
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     qq += __shfl_xor_sync(full, qq, o);
@@ -245,7 +264,7 @@ __device__ Cut topm_cut(const float* __restrict__ row, int c, int m, int* hist, 
   cut.cutJ = 0x7fffffff;
   int a = 0, nc = 0;
   for (int j = lane; j < c; j += 32) {
-    const double s = (double)row[j];
+    const double s = (double)ldf<kCoh>(row + j);
     a += s > cut.hi;
     nc += (s >= cut.lo && s <= cut.hi);
   }
@@ -266,7 +285,7 @@ __device__ Cut topm_cut(const float* __restrict__ row, int c, int m, int* hist, 
       const int j = j0 + lane;
       bool inb = false;
       if (j < c) {
-        const double s = (double)row[j];
+        const double s = (double)ldf<kCoh>(row + j);
         inb = s >= cut.lo && s <= cut.hi;
       }
       const unsigned bb = __ballot_sync(full, inb);
@@ -279,7 +298,7 @@ __device__ Cut topm_cut(const float* __restrict__ row, int c, int m, int* hist, 
     double my_e = -INFINITY;
     int my_key_j = 0x7fffffff;
     if (my_j >= 0) {
-      my_e = exact_score(qrow, Kp + (kv_row0 + my_j) * kHeadDim);
+      my_e = exact_score<kCoh>(qrow, Kp + (kv_row0 + my_j) * kHeadDim);
       my_key_j = my_j;
     }
 #pragma unroll
@@ -308,9 +327,9 @@ __device__ Cut topm_cut(const float* __restrict__ row, int c, int m, int* hist, 
       double be = -INFINITY;
       int bj = 0x7fffffff;
       for (int j = lane; j < c; j += 32) {
-        const double s = (double)row[j];
+        const double s = (double)ldf<kCoh>(row + j);
         if (s < cut.lo || s > cut.hi) continue;
-        const double e = exact_score(qrow, Kp + (kv_row0 + j) * kHeadDim);
+        const double e = exact_score<kCoh>(qrow, Kp + (kv_row0 + j) * kHeadDim);
         if (ranks_above(pe, pj, e, j) && ranks_above(e, j, be, bj)) {
           be = e;
           bj = j;
@@ -335,16 +354,18 @@ __device__ Cut topm_cut(const float* __restrict__ row, int c, int m, int* hist, 
 }
 
 // Is candidate j (fp32 score s) inside the exact top-m described by `cut`?
+template <bool kCoh>
 __device__ __forceinline__ bool in_cut(const Cut& cut, float s32, int j, const float* __restrict__ qrow,
                                        const float* __restrict__ Kp, long long kv_row0) {
   const double s = (double)s32;
   if (s > cut.hi) return true;
   if (s < cut.lo) return false;
-  return cut.all_band || !ranks_above(cut.cutE, cut.cutJ, exact_score(qrow, Kp + (kv_row0 + j) * kHeadDim), j);
+  return cut.all_band || !ranks_above(cut.cutE, cut.cutJ, exact_score<kCoh>(qrow, Kp + (kv_row0 + j) * kHeadDim), j);
 }
 
 // one warp: the top-k row wr of the head batch starting at head bh0 (hist:
 // this warp's 256 ints of shared scratch)
+template <bool kCoh>
 __device__ __forceinline__ void select_row(const float* __restrict__ Qp, const float* __restrict__ Kp,
                                            const float* __restrict__ kn, int Hq, int G, int Nmax,
                                            const int32_t* __restrict__ n_chunks, int k, int stride, long long bh0,
@@ -356,7 +377,7 @@ __device__ __forceinline__ void select_row(const float* __restrict__ Qp, const f
   const int i = (int)(wr % Nmax);
   const long long bh = bh0 + bhl;
   const int b = (int)(bh / Hq), hq = (int)(bh % Hq);
-  const int n = n_chunks[b];
+  const int n = min(max(n_chunks[b], 0), Nmax);   // a count outside [0, Nmax] is clamped
   int32_t* out = sel + (bh * Nmax + i) * stride;
   int cnt = 0;
   if (i < n) {
@@ -368,12 +389,12 @@ __device__ __forceinline__ void select_row(const float* __restrict__ Qp, const f
       const float* row = ws + bhl * tri(Nmax) + tri(i);
       const long long kv_row0 = ((long long)b * (Hq / G) + hq / G) * Nmax;
       const float* qrow = Qp + (bh * Nmax + i) * kHeadDim;
-      const Cut cut = topm_cut(row, i, m, hist, qrow, Kp, kv_row0, kn);
+      const Cut cut = topm_cut<kCoh>(row, i, m, hist, qrow, Kp, kv_row0, kn);
       // --- output, ascending
       int written = 0;
       for (int j0 = 0; j0 < i; j0 += 32) {
         const int j = j0 + lane;
-        const bool take = j < i && in_cut(cut, row[j], j, qrow, Kp, kv_row0);
+        const bool take = j < i && in_cut<kCoh>(cut, ldf<kCoh>(row + j), j, qrow, Kp, kv_row0);
         const unsigned bt = __ballot_sync(full, take);
         const int pos = written + __popc(bt & lanemask_lt());
         if (take && pos < m) out[pos] = j;
@@ -397,7 +418,7 @@ __global__ void __launch_bounds__(256) select_kernel(const float* __restrict__ Q
   __shared__ int hist_all[8][256];
   const int warp = threadIdx.x >> 5;
   const long long wr = (long long)blockIdx.x * 8 + warp;      // row within the head batch
-  if (wr < n_rows) select_row(Qp, Kp, kn, Hq, G, Nmax, n_chunks, k, stride, bh0, wr, ws, sel, n_sel, hist_all[warp]);
+  if (wr < n_rows) select_row<false>(Qp, Kp, kn, Hq, G, Nmax, n_chunks, k, stride, bh0, wr, ws, sel, n_sel, hist_all[warp]);
 }
 
 // ------------------------------------------------------------------ 3'. row budgets
@@ -427,7 +448,7 @@ __global__ void __launch_bounds__(256) budget_select_kernel(
   const int i = (int)(wr % Nmax);
   const long long bh = bh0 + bhl;
   const int b = (int)(bh / Hq), hq = (int)(bh % Hq);
-  const int n = n_chunks[b];
+  const int n = min(max(n_chunks[b], 0), Nmax);   // a count outside [0, Nmax] is clamped
   int32_t* out = sel + (bh * Nmax + i) * stride;
   int* hist = hist_all[warp];
   int* mj = mj_all[warp];
@@ -448,12 +469,12 @@ __global__ void __launch_bounds__(256) budget_select_kernel(
       const float* qrow = Qp + (bh * Nmax + i) * kHeadDim;
       const bool all = (m == c);
       Cut cut{};
-      if (!all) cut = topm_cut(row, c, m, hist, qrow, Kp, kv_row0, kn);
+      if (!all) cut = topm_cut<false>(row, c, m, hist, qrow, Kp, kv_row0, kn);
       // members of the top m, ascending index
       int nm = 0;
       for (int j0 = 0; j0 < c; j0 += 32) {
         const int j = j0 + lane;
-        const bool take = j < c && (all || in_cut(cut, row[j], j, qrow, Kp, kv_row0));
+        const bool take = j < c && (all || in_cut<false>(cut, row[j], j, qrow, Kp, kv_row0));
         const unsigned bt = __ballot_sync(full, take);
         const int pos = nm + __popc(bt & lanemask_lt());
         if (take && pos < m) mj[pos] = j;
@@ -461,7 +482,7 @@ __global__ void __launch_bounds__(256) budget_select_kernel(
       }
       nm = min(nm, m);
       __syncwarp();
-      for (int a = lane; a < nm; a += 32) me[a] = exact_score(qrow, Kp + (kv_row0 + mj[a]) * kHeadDim);
+      for (int a = lane; a < nm; a += 32) me[a] = exact_score<false>(qrow, Kp + (kv_row0 + mj[a]) * kHeadDim);
       __syncwarp();
       // rank of each member; lengths in rank order
       for (int a = lane; a < nm; a += 32) {
@@ -523,7 +544,10 @@ long long heads_per_batch(int B, int Hq, int Nmax) {
 // per-block code as its separate kernel, so the results are bit-identical.
 struct GridBar {
   unsigned int* count;    // arrivals so far (zeroed before the launch)
+  unsigned int* abort;    // set by a block that gave up waiting (zeroed before the launch)
   unsigned int* status;
+  unsigned long long limit_ns;   // wall-clock limit of one barrier wait
+  unsigned long long hold_ns;    // test hook: block 0 arrives this late at the first barrier (0: off)
 };
 
 __device__ __forceinline__ unsigned ld_acquire_u32(const unsigned int* p) {
@@ -532,26 +556,44 @@ __device__ __forceinline__ unsigned ld_acquire_u32(const unsigned int* p) {
   return v;
 }
 
-// Every block arrives once per barrier; thread 0 waits until all have, and
-// gives up after 1 s of wall-clock time (DHSA_DEVFLAG_WAIT_TIMEOUT).
-__device__ __forceinline__ void grid_barrier(const GridBar& gb, unsigned& phase) {
+// Every block arrives once per barrier; thread 0 waits until all have. A wait
+// that passes limit_ns raises DHSA_DEVFLAG_WAIT_TIMEOUT and the abort word;
+// a block that sees the abort word stops waiting. Either way the barrier
+// returns false and the block leaves the kernel (the phases after it would
+// read unfinished results). Returns true once every block has arrived.
+__device__ __forceinline__ bool grid_barrier(const GridBar& gb, unsigned& phase) {
+  __shared__ int s_ok;
   __syncthreads();
   ++phase;
   if (threadIdx.x == 0) {
+    int ok = 1;
+    if (gb.hold_ns && phase == 1 && blockIdx.x == 0) {
+      // test hook: arrive late (bounded), or as soon as another block gave up
+      const uint64_t t0 = ptx::globaltimer_ns();
+      while (ptx::globaltimer_ns() - t0 < gb.hold_ns && ld_acquire_u32(gb.abort) == 0u) __nanosleep(256);
+    }
     __threadfence();
     atomicAdd(gb.count, 1u);
     const unsigned target = phase * gridDim.x;
     const uint64_t t0 = ptx::globaltimer_ns();
     while (ld_acquire_u32(gb.count) < target) {
-      if (ptx::globaltimer_ns() - t0 > 1000000000ull) {
+      if (ld_acquire_u32(gb.abort) != 0u) {
+        ok = 0;
+        break;
+      }
+      if (ptx::globaltimer_ns() - t0 > gb.limit_ns) {
+        atomicExch(gb.abort, 1u);
         raise_device_flag(gb.status, DHSA_DEVFLAG_WAIT_TIMEOUT);
+        ok = 0;
         break;
       }
       __nanosleep(64);
     }
     __threadfence();
+    s_ok = ok;
   }
   __syncthreads();
+  return s_ok != 0;
 }
 
 constexpr int kFusedKC = 2;   // 64-key score tiles in the fused kernel: three blocks per SM
@@ -572,12 +614,12 @@ __global__ void __launch_bounds__(256, 3) route_fused_kernel(const uint4* __rest
   // pooled Q and K rows
   const long long rows_q = (long long)B * Hq * Nmax, rows_k = (long long)B * Hkv * Nmax;
   for (long long w = gwarp; w < rows_q + rows_k; w += nwarps) {
-    if (w < rows_q) pool_row(Q, Hq, L, off, n_chunks, Nmax, w, Qp);
-    else pool_row(K, Hkv, L, off, n_chunks, Nmax, w - rows_q, Kp);
+    if (w < rows_q) pool_row(Q, Hq, L, off, n_chunks, Nmax, w, Qp, gb.status);
+    else pool_row(K, Hkv, L, off, n_chunks, Nmax, w - rows_q, Kp, gb.status);
   }
-  grid_barrier(gb, phase);
+  if (!grid_barrier(gb, phase)) return;
   // key norms (read by the selection only) and the score tiles of each head batch
-  for (long long r = gwarp; r < rows_k; r += nwarps) key_norm_row(Kp, r, kn);
+  for (long long r = gwarp; r < rows_k; r += nwarps) key_norm_row<true>(Kp, r, kn);
   const int n_rb = (Nmax + TR - 1) / TR, n_kb = (Nmax + 32 * kFusedKC - 1) / (32 * kFusedKC);
   const long long total = (long long)B * Hq;
   int* hist = reinterpret_cast<int*>(sm) + (threadIdx.x >> 5) * 256;
@@ -586,13 +628,13 @@ __global__ void __launch_bounds__(256, 3) route_fused_kernel(const uint4* __rest
     const long long tiles = nh * n_rb * n_kb;
     for (long long t = blockIdx.x; t < tiles; t += gridDim.x) {
       const int bhl = (int)(t / (n_rb * n_kb)), rest = (int)(t % (n_rb * n_kb));
-      score_tile_body<kFusedKC>(Qp, Kp, Hq, G, Nmax, n_chunks, h0, bhl, rest / n_kb, rest % n_kb, scores, sm);
+      score_tile_body<kFusedKC, true>(Qp, Kp, Hq, G, Nmax, n_chunks, h0, bhl, rest / n_kb, rest % n_kb, scores, sm);
       __syncthreads();   // the next tile restages shared memory
     }
-    grid_barrier(gb, phase);
+    if (!grid_barrier(gb, phase)) return;
     for (long long wr = gwarp; wr < nh * Nmax; wr += nwarps)
-      select_row(Qp, Kp, kn, Hq, G, Nmax, n_chunks, k, stride, h0, wr, scores, sel, n_sel, hist);
-    if (h0 + hb < total) grid_barrier(gb, phase);   // the next head batch overwrites the scores
+      select_row<true>(Qp, Kp, kn, Hq, G, Nmax, n_chunks, k, stride, h0, wr, scores, sel, n_sel, hist);
+    if (h0 + hb < total && !grid_barrier(gb, phase)) return;   // the next head batch overwrites the scores
   }
 }
 
@@ -637,10 +679,13 @@ int launch_score_topk(const float* Qp, const float* Kp, int B, int Hq, int Hkv, 
 }
 
 // All of routing up to the selection in one cooperative launch (workspace as
-// for launch_score_topk; its first 4 bytes hold the grid barrier's counter).
+// for launch_score_topk; its first 8 bytes hold the grid barrier's counter
+// and abort word). limit_ns bounds each barrier wait; hold_ns > 0 is the test
+// hook that makes block 0 arrive late at the first barrier.
 int launch_route_fused(const void* Q, const void* K, int B, int Hq, int Hkv, int L, const int32_t* off,
                        const int32_t* n_chunks, int Nmax, int k, float* Qp, float* Kp, int32_t* sel, int32_t* n_sel,
-                       void* ws, unsigned int* status, cudaStream_t stream) {
+                       void* ws, unsigned int* status, unsigned long long limit_ns, unsigned long long hold_ns,
+                       cudaStream_t stream) {
   const int stride = score_topk_stride(k, Nmax);
   float* kn = reinterpret_cast<float*>(static_cast<char*>(ws) + 256);
   const size_t kn_bytes = (sizeof(float) * (size_t)B * Hq * Nmax + 255) & ~size_t(255);
@@ -652,10 +697,10 @@ int launch_route_fused(const void* Q, const void* K, int B, int Hq, int Hkv, int
   if (e == cudaSuccess) e = cudaGetDevice(&dev);
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, route_fused_kernel, 256, smem);
-  if (e == cudaSuccess) e = cudaMemsetAsync(ws, 0, sizeof(unsigned int), stream);
+  if (e == cudaSuccess) e = cudaMemsetAsync(ws, 0, 2 * sizeof(unsigned int), stream);
   if (e != cudaSuccess) return cuda_status(e);
   if (per_sm < 1) return DHSA_ERR_UNSUPPORTED;
-  GridBar gb{static_cast<unsigned int*>(ws), status};
+  GridBar gb{static_cast<unsigned int*>(ws), static_cast<unsigned int*>(ws) + 1, status, limit_ns, hold_ns};
   const uint4* q4 = static_cast<const uint4*>(Q);
   const uint4* k4 = static_cast<const uint4*>(K);
   void* args[] = {(void*)&q4,     (void*)&k4,   (void*)&B,     (void*)&Hq,   (void*)&Hkv,   (void*)&L,

@@ -118,3 +118,12 @@ def test_fused_routing_arguments_rejected_on_host(lib):
     assert f(FAKE, FAKE, 1, 4, 2, 64, 96, FAKE, FAKE, 8, 2, FAKE, FAKE, FAKE, FAKE, FAKE, ws, None) == UNS
     assert f(FAKE, FAKE, 1, 4, 2, 64, 128, FAKE, FAKE, 8, 2, FAKE, FAKE, FAKE, FAKE, None, ws, None) == WS
     assert f(FAKE, FAKE, 1, 4, 2, 64, 128, FAKE, FAKE, 8, 2, FAKE, FAKE, FAKE, FAKE, FAKE, ws - 16, None) == WS
+
+
+def test_wait_timeout_hook_arguments(lib):
+    # host-side only: arming records state for the next launch; bad values are refused
+    assert lib.dhsa_debug_arm_wait_timeout(3, 1000) == 1
+    assert lib.dhsa_debug_arm_wait_timeout(1, 0) == 1
+    assert lib.dhsa_debug_arm_wait_timeout(2, 10 ** 9) == 1
+    assert lib.dhsa_debug_arm_wait_timeout(1, 50_000) == 0
+    assert lib.dhsa_debug_arm_wait_timeout(0, 0) == 0

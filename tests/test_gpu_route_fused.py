@@ -29,6 +29,11 @@ CASES = {
     "short-seq": I.custom(B=3, Hq=2, Hkv=1, L=37, lo=1, hi=9, k=2, wid=107),
     "geometric": I.custom(B=2, Hq=4, Hkv=1, L=3000, lo=1, hi=1024, kind="geometric", mean=40.0, k=6, wid=108),
     "many-chunks": I.custom(B=1, Hq=2, Hkv=1, L=16000, lo=1, hi=3, k=5, wid=120),
+    # ~12000 chunks: one head's packed scores (~288 MB) exceed the 256 MiB
+    # score workspace, so the four heads run as four head batches, with a
+    # grid barrier between a batch's selection and the next batch's score
+    # tiles overwriting the same scores
+    "four-head-batches": I.custom(B=1, Hq=4, Hkv=1, L=24000, lo=1, hi=3, k=5, wid=122),
     "llama8b-32k": I.WORKLOADS["llama8b-32k"],
 }
 
