@@ -173,6 +173,19 @@ int dhsa_chunk_score_select_budget(const float* Qp, const float* Kp, int B, int 
                                    const int32_t* budgets, int recent, int k_max, int32_t* sel, int32_t* n_sel,
                                    void* workspace, size_t workspace_bytes, void* stream);
 
+/* 2b. Similarity and top-k as in 2., writing the block CSR of 3. as well.
+ *    Under the top-k rule row i < n_chunks[b] keeps min(k, i) + 1 chunks, so
+ *    every row's CSR offset has a closed form and each selection row writes
+ *    its CSR row directly (no scan, no second pass over sel). Results equal
+ *    dhsa_chunk_score_topk followed by dhsa_build_block_csr, bit for bit:
+ *    sel and n_sel as in 2., row_ptr / col_idx / cost (nullable) as in 3.
+ *    (col_idx needs dhsa_csr_nnz_upper(B, Hq, Nmax, k) entries). off is the
+ *    offsets table of 1. Workspace and errors as for 2. */
+int dhsa_chunk_score_topk_csr(const float* Qp, const float* Kp, int B, int Hq, int Hkv, int Nmax,
+                              const int32_t* off, const int32_t* n_chunks, int k, int32_t* sel, int32_t* n_sel,
+                              int32_t* row_ptr, int32_t* col_idx, int64_t* cost, void* workspace,
+                              size_t workspace_bytes, void* stream);
+
 /* ---------------------------------------------------------------------------
  * 2c. Pooling, similarity and top-k in one launch.
  *    Sources as for 1. and 2.; the gist.science technical summary places the
@@ -185,7 +198,9 @@ int dhsa_chunk_score_select_budget(const float* Qp, const float* Kp, int B, int 
  *    barrier sets DHSA_DEVFLAG_WAIT_TIMEOUT and an abort word, and every
  *    block then leaves the kernel; the outputs of that launch are undefined).
  *    Arguments and layouts are those of the two calls; Qp and Kp are written
- *    as by 1b.
+ *    as by 1b. On B200 the separate launches are faster (they keep more
+ *    warps in flight for the HBM-bound pooling and the latency-bound
+ *    selection); this entry serves callers that want one launch.
  *    workspace: dhsa_route_fused_workspace_size(B, Hq, Nmax) bytes (equal to
  *    dhsa_score_topk_workspace_size; its first 8 bytes hold the barrier
  *    count and the abort word, reset by this call on `stream`). Calls
@@ -195,6 +210,15 @@ size_t dhsa_route_fused_workspace_size(int B, int Hq, int Nmax);
 int dhsa_route_fused(const void* Q, const void* K, int B, int Hq, int Hkv, int L, int head_dim, const int32_t* off,
                      const int32_t* n_chunks, int Nmax, int k, float* Qp, float* Kp, int32_t* sel, int32_t* n_sel,
                      void* workspace, size_t workspace_bytes, void* stream);
+
+/* 2d. The one launch of 2c. also writing the block CSR of 3., as 2b. does.
+ *    Results equal dhsa_route_fused followed by dhsa_build_block_csr, bit
+ *    for bit. row_ptr, col_idx and cost (nullable) as in 3.; other
+ *    arguments, the workspace and errors as for 2c. */
+int dhsa_route_topk_csr(const void* Q, const void* K, int B, int Hq, int Hkv, int L, int head_dim,
+                        const int32_t* off, const int32_t* n_chunks, int Nmax, int k, float* Qp, float* Kp,
+                        int32_t* sel, int32_t* n_sel, int32_t* row_ptr, int32_t* col_idx, int64_t* cost,
+                        void* workspace, size_t workspace_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
  * 3. Upsampling to the token keep-set, stored as a block CSR.
@@ -313,9 +337,9 @@ int dhsa_sparse_attn_fwd_tiles(const void* Q, const void* K, const void* V, int 
  *              which precedes every copy and MMA -- runs out after limit_ns;
  *              the CTAs record the flag, free their TMEM and return without
  *              writing O.
- *      mode 2: the next dhsa_route_fused launch has block 0 arrive late at
- *              its first grid barrier; the other blocks give up after
- *              limit_ns, set the abort word, and all blocks leave.
+ *      mode 2: the next one-launch routing (2c., 2d.) has block 0 arrive
+ *              late at its first grid barrier; the other blocks give up
+ *              after limit_ns, set the abort word, and all blocks leave.
  *      mode 0: disarm.
  *    The hook is one-shot (the launch that uses it disarms it) and host-side
  *    state of the library: not thread-safe, for tests only.

@@ -50,10 +50,13 @@ _SIGNATURES = {
     "dhsa_sel_stride": (_I, [_I, _I]),
     "dhsa_score_topk_workspace_size": (_SZ, [_I, _I, _I]),
     "dhsa_chunk_score_topk": (_I, [_P, _P, _I, _I, _I, _I, _P, _I, _P, _P, _P, _SZ, _P]),
+    "dhsa_chunk_score_topk_csr": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, _I, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "dhsa_budget_max_chunks": (_I, []),
     "dhsa_chunk_score_select_budget": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, _I, _P, _I, _I, _P, _P, _P, _SZ, _P]),
     "dhsa_route_fused_workspace_size": (_SZ, [_I, _I, _I]),
     "dhsa_route_fused": (_I, [_P, _P, _I, _I, _I, _I, _I, _P, _P, _I, _I, _P, _P, _P, _P, _P, _SZ, _P]),
+    "dhsa_route_topk_csr": (_I, [_P, _P, _I, _I, _I, _I, _I, _P, _P, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _SZ,
+                                 _P]),
     "dhsa_csr_nnz_upper": (_SZ, [_I, _I, _I, _I]),
     "dhsa_build_block_csr": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P]),
     "dhsa_sparse_attn_workspace_size": (_SZ, [_I, _I, _I, _I]),
@@ -181,6 +184,36 @@ def sel_stride(k: int, nmax: int) -> int:
     return load().dhsa_sel_stride(k, nmax)
 
 
+def chunk_score_topk_csr(Qp: torch.Tensor, Kp: torch.Tensor, off: torch.Tensor, n_chunks: torch.Tensor, k: int,
+                         sel: torch.Tensor, n_sel: torch.Tensor, row_ptr: torch.Tensor, col_idx: torch.Tensor,
+                         cost: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None):
+    """Top-k selection that also writes the block CSR (include/dhsa.h, 2b):
+    the results of chunk_score_topk followed by build_block_csr."""
+    B, Hq, nmax, d = Qp.shape
+    Hkv = Kp.shape[1]
+    _need(Qp, torch.float32, None, "Qp")
+    _need(Kp, torch.float32, (B, Hkv, nmax, d), "Kp")
+    _need(off, torch.int32, (B, nmax + 1), "off")
+    _need(n_chunks, torch.int32, (B,), "n_chunks")
+    lib = load()
+    stride = lib.dhsa_sel_stride(k, nmax)
+    _need(sel, torch.int32, (B, Hq, nmax, stride), "sel")
+    _need(n_sel, torch.int32, (B, Hq, nmax), "n_sel")
+    _need(row_ptr, torch.int32, (B * Hq * nmax + 1,), "row_ptr")
+    _need(col_idx, torch.int32, None, "col_idx")
+    if col_idx.numel() < lib.dhsa_csr_nnz_upper(B, Hq, nmax, k):
+        raise ValueError("col_idx: smaller than dhsa_csr_nnz_upper")
+    if cost is not None:
+        _need(cost, torch.int64, (B * Hq * nmax,), "cost")
+    if workspace is None:
+        workspace = torch.empty(lib.dhsa_score_topk_workspace_size(B, Hq, nmax), dtype=torch.uint8, device=Qp.device)
+    _check(lib.dhsa_chunk_score_topk_csr(_ptr(Qp), _ptr(Kp), B, Hq, Hkv, nmax, _ptr(off), _ptr(n_chunks), k,
+                                         _ptr(sel), _ptr(n_sel), _ptr(row_ptr), _ptr(col_idx), _ptr(cost),
+                                         _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                         _stream_ptr()), "dhsa_chunk_score_topk_csr")
+    return sel, n_sel
+
+
 def chunk_score_topk(Qp: torch.Tensor, Kp: torch.Tensor, n_chunks: torch.Tensor, k: int,
                      sel: Optional[torch.Tensor] = None, n_sel: Optional[torch.Tensor] = None,
                      workspace: Optional[torch.Tensor] = None):
@@ -211,10 +244,12 @@ def chunk_score_topk(Qp: torch.Tensor, Kp: torch.Tensor, n_chunks: torch.Tensor,
 def route_fused(Q: torch.Tensor, K: torch.Tensor, off: torch.Tensor, n_chunks: torch.Tensor, k: int,
                 Qp: Optional[torch.Tensor] = None, Kp: Optional[torch.Tensor] = None,
                 sel: Optional[torch.Tensor] = None, n_sel: Optional[torch.Tensor] = None,
-                workspace: Optional[torch.Tensor] = None):
+                workspace: Optional[torch.Tensor] = None, row_ptr: Optional[torch.Tensor] = None,
+                col_idx: Optional[torch.Tensor] = None, cost: Optional[torch.Tensor] = None):
     """Pooling of Q and K plus the top-k selection in one launch (include/dhsa.h,
-    2c); the same results as chunk_pool_qk followed by chunk_score_topk.
-    Returns (Qp, Kp, sel, n_sel)."""
+    2c); the same results as chunk_pool_qk followed by chunk_score_topk. With
+    row_ptr and col_idx given, the launch also writes the block CSR (2d), as
+    build_block_csr would. Returns (Qp, Kp, sel, n_sel)."""
     B, Hq, L, d = Q.shape
     Hkv = K.shape[1]
     nmax = off.shape[1] - 1
@@ -239,9 +274,21 @@ def route_fused(Q: torch.Tensor, K: torch.Tensor, off: torch.Tensor, n_chunks: t
     ws_bytes = lib.dhsa_route_fused_workspace_size(B, Hq, nmax)
     if workspace is None:
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=Q.device)
-    _check(lib.dhsa_route_fused(_ptr(Q), _ptr(K), B, Hq, Hkv, L, d, _ptr(off), _ptr(n_chunks), nmax, k, _ptr(Qp),
-                                _ptr(Kp), _ptr(sel), _ptr(n_sel), _ptr(workspace),
-                                workspace.numel() * workspace.element_size(), _stream_ptr()), "dhsa_route_fused")
+    if row_ptr is None:
+        _check(lib.dhsa_route_fused(_ptr(Q), _ptr(K), B, Hq, Hkv, L, d, _ptr(off), _ptr(n_chunks), nmax, k,
+                                    _ptr(Qp), _ptr(Kp), _ptr(sel), _ptr(n_sel), _ptr(workspace),
+                                    workspace.numel() * workspace.element_size(), _stream_ptr()), "dhsa_route_fused")
+    else:
+        _need(row_ptr, torch.int32, (B * Hq * nmax + 1,), "row_ptr")
+        _need(col_idx, torch.int32, None, "col_idx")
+        if col_idx.numel() < lib.dhsa_csr_nnz_upper(B, Hq, nmax, k):
+            raise ValueError("col_idx: smaller than dhsa_csr_nnz_upper")
+        if cost is not None:
+            _need(cost, torch.int64, (B * Hq * nmax,), "cost")
+        _check(lib.dhsa_route_topk_csr(_ptr(Q), _ptr(K), B, Hq, Hkv, L, d, _ptr(off), _ptr(n_chunks), nmax, k,
+                                       _ptr(Qp), _ptr(Kp), _ptr(sel), _ptr(n_sel), _ptr(row_ptr), _ptr(col_idx),
+                                       _ptr(cost), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                       _stream_ptr()), "dhsa_route_topk_csr")
     return Qp, Kp, sel, n_sel
 
 
@@ -365,19 +412,22 @@ class DHSAPrefill:
     a window of `recent` chunks and at most k earlier chunks per row.
     `short_tiles` picks the query-tile policy of the attention (0: 128-row
     tiles only, the fast default; 1 and 2: see sparse_attn_fwd).
-    `fused_routing` runs pooling and the top-k selection as one launch
-    (route_fused; top-k rule only).
+    `fused_routing` runs pooling, the top-k selection and the CSR as one
+    launch (route_fused; top-k rule only). Under the top-k rule the selection
+    writes the CSR itself (chunk_score_topk_csr); `csr_from_selection=False`
+    runs the separate CSR build instead (the same results).
     """
 
     def __init__(self, B: int, Hq: int, Hkv: int, L: int, off: torch.Tensor, n_chunks: torch.Tensor, k: int,
                  device="cuda", softmax_scale: Optional[float] = None, budget=None, recent: int = 0,
-                 short_tiles: int = 0, fused_routing: bool = False):
+                 short_tiles: int = 0, fused_routing: bool = False, csr_from_selection: bool = True):
         lib = load()
         self.B, self.Hq, self.Hkv, self.L, self.k = B, Hq, Hkv, L, k
         self.short_tiles = short_tiles
         if fused_routing and budget is not None:
             raise ValueError("fused_routing supports the top-k rule only")
         self.fused_routing = fused_routing
+        self.csr_from_selection = csr_from_selection
         self.budget, self.recent = budget, recent
         self.off, self.n_chunks = off, n_chunks
         self.nmax = off.shape[1] - 1
@@ -401,11 +451,14 @@ class DHSAPrefill:
     def routing(self, Q, K):
         if self.fused_routing:
             route_fused(Q, K, self.off, self.n_chunks, self.k, Qp=self.Qp, Kp=self.Kp, sel=self.sel,
-                        n_sel=self.n_sel, workspace=self.ws_topk)
-            build_block_csr(self.sel, self.n_sel, self.k, self.off, self.n_chunks, row_ptr=self.row_ptr,
-                            col_idx=self.col_idx, cost=self.cost)
+                        n_sel=self.n_sel, workspace=self.ws_topk, row_ptr=self.row_ptr, col_idx=self.col_idx,
+                        cost=self.cost)
             return
         chunk_pool_qk(Q, K, self.off, self.n_chunks, Qp=self.Qp, Kp=self.Kp)
+        if self.budget is None and self.csr_from_selection:
+            chunk_score_topk_csr(self.Qp, self.Kp, self.off, self.n_chunks, self.k, self.sel, self.n_sel,
+                                 self.row_ptr, self.col_idx, cost=self.cost, workspace=self.ws_topk)
+            return
         if self.budget is None:
             chunk_score_topk(self.Qp, self.Kp, self.n_chunks, self.k, sel=self.sel, n_sel=self.n_sel,
                              workspace=self.ws_topk)

@@ -16,11 +16,11 @@ int launch_validate_offsets(const int32_t* off, const int32_t* n_chunks, int B, 
 int score_topk_stride(int k, int Nmax);
 size_t score_topk_ws_bytes(int B, int Hq, int Nmax);
 int launch_score_topk(const float* Qp, const float* Kp, int B, int Hq, int Hkv, int Nmax, const int32_t* n_chunks,
-                      int k, int32_t* sel, int32_t* n_sel, void* ws, cudaStream_t stream);
+                      int k, int32_t* sel, int32_t* n_sel, void* ws, const CsrOut& csr, cudaStream_t stream);
 int launch_route_fused(const void* Q, const void* K, int B, int Hq, int Hkv, int L, const int32_t* off,
                        const int32_t* n_chunks, int Nmax, int k, float* Qp, float* Kp, int32_t* sel, int32_t* n_sel,
-                       void* ws, unsigned int* status, unsigned long long limit_ns, unsigned long long hold_ns,
-                       cudaStream_t stream);
+                       const CsrOut& csr, void* ws, unsigned int* status, unsigned long long limit_ns,
+                       unsigned long long hold_ns, cudaStream_t stream);
 int score_budget_max_chunks();
 int launch_score_budget(const float* Qp, const float* Kp, int B, int Hq, int Hkv, int Nmax, const int32_t* off,
                         const int32_t* n_chunks, int budget, const int32_t* budgets, int recent, int k_max,
@@ -194,10 +194,29 @@ int dhsa_chunk_score_topk(const float* Qp, const float* Kp, int B, int Hq, int H
   if (!Qp || !Kp || !n_chunks || !sel || !n_sel) return DHSA_ERR_INVALID_ARG;
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || Nmax <= 0 || k < 0 || Hq % Hkv != 0) return DHSA_ERR_INVALID_ARG;
   const size_t need = score_topk_ws_bytes(B, Hq, Nmax);
-  if (need && (!workspace || workspace_bytes < need || !aligned16(workspace))) return DHSA_ERR_WORKSPACE;
+  if (!workspace || workspace_bytes < need || !aligned16(workspace)) return DHSA_ERR_WORKSPACE;
   int st = check_device_sm100();
   if (st != DHSA_OK) return st;
-  return launch_score_topk(Qp, Kp, B, Hq, Hkv, Nmax, n_chunks, k, sel, n_sel, need ? workspace : nullptr,
+  const CsrOut none{nullptr, nullptr, nullptr, nullptr, nullptr};
+  return launch_score_topk(Qp, Kp, B, Hq, Hkv, Nmax, n_chunks, k, sel, n_sel, workspace, none,
+                           static_cast<cudaStream_t>(stream));
+}
+
+int dhsa_chunk_score_topk_csr(const float* Qp, const float* Kp, int B, int Hq, int Hkv, int Nmax,
+                              const int32_t* off, const int32_t* n_chunks, int k, int32_t* sel, int32_t* n_sel,
+                              int32_t* row_ptr, int32_t* col_idx, int64_t* cost, void* workspace,
+                              size_t workspace_bytes, void* stream) {
+  if (!Qp || !Kp || !off || !n_chunks || !sel || !n_sel || !row_ptr || !col_idx) return DHSA_ERR_INVALID_ARG;
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Nmax <= 0 || k < 0 || Hq % Hkv != 0) return DHSA_ERR_INVALID_ARG;
+  if (dhsa_csr_nnz_upper(B, Hq, Nmax, k) > 0x7fffffffULL) return DHSA_ERR_INVALID_ARG;   // int32 row_ptr
+  const size_t need = score_topk_ws_bytes(B, Hq, Nmax);
+  if (!workspace || workspace_bytes < need || !aligned16(workspace)) return DHSA_ERR_WORKSPACE;
+  int st = check_device_sm100();
+  if (st != DHSA_OK) return st;
+  unsigned int* status = device_status_ptr();
+  if (!status) return DHSA_ERR_CUDA;
+  const CsrOut csr{row_ptr, col_idx, cost, off, status};
+  return launch_score_topk(Qp, Kp, B, Hq, Hkv, Nmax, n_chunks, k, sel, n_sel, workspace, csr,
                            static_cast<cudaStream_t>(stream));
 }
 
@@ -206,9 +225,11 @@ size_t dhsa_route_fused_workspace_size(int B, int Hq, int Nmax) {
   return score_topk_ws_bytes(B, Hq, Nmax);
 }
 
-int dhsa_route_fused(const void* Q, const void* K, int B, int Hq, int Hkv, int L, int head_dim, const int32_t* off,
-                     const int32_t* n_chunks, int Nmax, int k, float* Qp, float* Kp, int32_t* sel, int32_t* n_sel,
-                     void* workspace, size_t workspace_bytes, void* stream) {
+namespace {
+int route_fused_common(const void* Q, const void* K, int B, int Hq, int Hkv, int L, int head_dim, const int32_t* off,
+                       const int32_t* n_chunks, int Nmax, int k, float* Qp, float* Kp, int32_t* sel, int32_t* n_sel,
+                       int32_t* row_ptr, int32_t* col_idx, int64_t* cost, void* workspace, size_t workspace_bytes,
+                       void* stream) {
   int st = check_layout(B, Hq, L, Nmax, off, n_chunks);
   if (st != DHSA_OK) return st;
   if (Hkv <= 0 || Hq % Hkv != 0 || k < 0) return DHSA_ERR_INVALID_ARG;
@@ -226,8 +247,28 @@ int dhsa_route_fused(const void* Q, const void* K, int B, int Hq, int Hkv, int L
     limit_ns = test_ns;
     hold_ns = 4 * test_ns + 1000000ull;
   }
-  return launch_route_fused(Q, K, B, Hq, Hkv, L, off, n_chunks, Nmax, k, Qp, Kp, sel, n_sel, workspace, status,
+  const CsrOut csr{row_ptr, col_idx, cost, off, status};
+  return launch_route_fused(Q, K, B, Hq, Hkv, L, off, n_chunks, Nmax, k, Qp, Kp, sel, n_sel, csr, workspace, status,
                             limit_ns, hold_ns, static_cast<cudaStream_t>(stream));
+}
+}  // namespace
+
+int dhsa_route_fused(const void* Q, const void* K, int B, int Hq, int Hkv, int L, int head_dim, const int32_t* off,
+                     const int32_t* n_chunks, int Nmax, int k, float* Qp, float* Kp, int32_t* sel, int32_t* n_sel,
+                     void* workspace, size_t workspace_bytes, void* stream) {
+  return route_fused_common(Q, K, B, Hq, Hkv, L, head_dim, off, n_chunks, Nmax, k, Qp, Kp, sel, n_sel, nullptr,
+                            nullptr, nullptr, workspace, workspace_bytes, stream);
+}
+
+int dhsa_route_topk_csr(const void* Q, const void* K, int B, int Hq, int Hkv, int L, int head_dim,
+                        const int32_t* off, const int32_t* n_chunks, int Nmax, int k, float* Qp, float* Kp,
+                        int32_t* sel, int32_t* n_sel, int32_t* row_ptr, int32_t* col_idx, int64_t* cost,
+                        void* workspace, size_t workspace_bytes, void* stream) {
+  if (!row_ptr || !col_idx) return DHSA_ERR_INVALID_ARG;
+  if (B > 0 && Hq > 0 && Nmax > 0 && k >= 0 && dhsa_csr_nnz_upper(B, Hq, Nmax, k) > 0x7fffffffULL)
+    return DHSA_ERR_INVALID_ARG;   // int32 row_ptr
+  return route_fused_common(Q, K, B, Hq, Hkv, L, head_dim, off, n_chunks, Nmax, k, Qp, Kp, sel, n_sel, row_ptr,
+                            col_idx, cost, workspace, workspace_bytes, stream);
 }
 
 int dhsa_budget_max_chunks(void) { return score_budget_max_chunks(); }

@@ -45,4 +45,13 @@ int check_device_sm100();
 
 __host__ __device__ inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
+// Block CSR written by the top-k selection itself (row_ptr null: none).
+struct CsrOut {
+  int32_t* row_ptr;
+  int32_t* col_idx;
+  int64_t* cost;        // may be null
+  const int32_t* off;
+  unsigned int* status;
+};
+
 }  // namespace dhsa

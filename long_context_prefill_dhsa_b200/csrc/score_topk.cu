@@ -68,32 +68,36 @@ __device__ __forceinline__ float4 ldf4(const float* p) {
 }
 
 // ------------------------------------------------------------------ 1. key norms
+// one warp: the norm of a 128-float row whose lane-th float4 is v (every
+// lane gets it); the fixed order makes every caller bit-identical
+__device__ __forceinline__ float warp_row_norm(const float4 v) {
+  double s = (double)v.x * v.x + (double)v.y * v.y + (double)v.z * v.z + (double)v.w * v.w;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  return (float)(sqrt(s) * (1.0 + 1e-6));   // fp32 rounding covered by the margin
+}
+
 // one warp: the norm of pooled key row r
 template <bool kCoh>
 __device__ __forceinline__ void key_norm_row(const float* __restrict__ Kp, long long r, float* __restrict__ kn) {
   const int lane = threadIdx.x & 31;
-  const float4 v = ldf4<kCoh>(Kp + r * kHeadDim + 4 * lane);
-  double s = (double)v.x * v.x + (double)v.y * v.y + (double)v.z * v.z + (double)v.w * v.w;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-  if (lane == 0) kn[r] = (float)(sqrt(s) * (1.0 + 1e-6));   // fp32 rounding covered by the margin
-}
-
-__global__ void __launch_bounds__(256) key_norm_kernel(const float* __restrict__ Kp, long long rows,
-                                                       float* __restrict__ kn) {
-  const long long r = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  if (r < rows) key_norm_row<false>(Kp, r, kn);
+  const float nrm = warp_row_norm(ldf4<kCoh>(Kp + r * kHeadDim + 4 * lane));
+  if (lane == 0) kn[r] = nrm;
 }
 
 // ------------------------------------------------------------------ 2. fp32 score tiles
 // one block: score tile (rb, kb) of head bh0 + bhl into that head's packed
 // rows of ws; a tile is TR query rows x 32 * KC keys (sm: TR * 128 +
 // 32 * KC * 132 floats of shared memory). Every score is one thread's fp32
-// dot product in a fixed order, whatever KC.
+// dot product in a fixed order, whatever KC. With kn given, the tiles of the
+// last row block of each kv group's first query head also write the norms
+// of their keys (computed from the staged rows exactly as key_norm_row does):
+// those tiles cover every key some row scores, once per kv head.
 template <int KC, bool kCoh>
 __device__ __forceinline__ void score_tile_body(const float* __restrict__ Qp, const float* __restrict__ Kp, int Hq,
                                                 int G, int Nmax, const int32_t* __restrict__ n_chunks, long long bh0,
-                                                int bhl, int rb, int kb, float* __restrict__ ws, float* sm) {
+                                                int bhl, int rb, int kb, float* __restrict__ ws, float* sm,
+                                                float* __restrict__ kn = nullptr) {
   float* Qs = sm;                        // [TR][128]
   float* Ks = sm + TR * kHeadDim;        // [32 * KC][132]
   const long long bh = bh0 + bhl;
@@ -119,6 +123,12 @@ __device__ __forceinline__ void score_tile_body(const float* __restrict__ Qp, co
   }
   __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (kn && hq % G == 0 && rb == (n - 1) / TR) {
+    for (int r = warp; r < 32 * KC && j0 + r < n; r += 8) {
+      const float nrm = warp_row_norm(*reinterpret_cast<const float4*>(Ks + r * kKsStride + 4 * lane));
+      if (lane == 0) kn[kv_row0 + j0 + r] = nrm;
+    }
+  }
   float acc[8][KC];
 #pragma unroll
   for (int r = 0; r < 8; ++r)
@@ -157,10 +167,11 @@ __device__ __forceinline__ void score_tile_body(const float* __restrict__ Qp, co
 __global__ void __launch_bounds__(256, 2) score_tile_kernel(const float* __restrict__ Qp,
                                                          const float* __restrict__ Kp, int Hq, int G, int Nmax,
                                                          const int32_t* __restrict__ n_chunks, long long bh0,
-                                                         int n_rb, int n_kb, float* __restrict__ ws) {
+                                                         int n_rb, int n_kb, float* __restrict__ ws,
+                                                         float* __restrict__ kn) {
   extern __shared__ __align__(16) float sm[];
   score_tile_body<TK / 32, false>(Qp, Kp, Hq, G, Nmax, n_chunks, bh0, blockIdx.y, blockIdx.x / n_kb, blockIdx.x % n_kb, ws,
-                          sm);
+                                  sm, kn);
 }
 
 // ------------------------------------------------------------------ 3. selection
@@ -409,16 +420,69 @@ __device__ __forceinline__ void select_row(const float* __restrict__ Qp, const f
   if (lane == 0) n_sel[bh * Nmax + i] = cnt;
 }
 
+// sum_{i < n} min(kk, i)
+__device__ __forceinline__ long long topk_prefix(long long n, long long kk) {
+  return n <= kk + 1 ? n * (n - 1) / 2 : kk * (kk + 1) / 2 + kk * (n - kk - 1);
+}
+
+// Block CSR of the top-k rule written straight from the selection. Under
+// that rule row i < n_b keeps min(k, i) + 1 chunks, so the CSR offset of a
+// row has a closed form: the rows before (b, hq, i) hold the sum over earlier
+// batch elements b' of Hq T(n_b'), plus hq T(n_b), plus i + F(i), with
+// F(i) = sum_{i' < i} min(k, i') and T(n) = n + F(n). Results equal the scan
+// and fill of csr.cu, bit for bit.
+// one warp: the CSR row of (bh, i) from its selection row (just written by
+// this warp; n_sel[bh * Nmax + i] holds its length)
+__device__ void csr_row(const CsrOut& o, const int32_t* sel, const int32_t* n_sel, const int32_t* n_chunks, int B,
+                        int Hq, int Nmax, int stride, long long bh, int i) {
+  const int lane = threadIdx.x & 31;
+  const int b = (int)(bh / Hq), hq = (int)(bh % Hq);
+  const long long kk = stride - 1;
+  long long base = 0;
+  for (int bb = 0; bb < b; ++bb) {
+    const long long nb = min(max(n_chunks[bb], 0), Nmax);
+    base += (long long)Hq * (nb + topk_prefix(nb, kk));
+  }
+  const long long n = min(max(n_chunks[b], 0), Nmax);
+  const long long T = n + topk_prefix(n, kk);
+  base += hq * T;
+  const long long rp = i < n ? base + i + topk_prefix(i, kk) : base + T;
+  const long long r = bh * Nmax + i;
+  const int cnt = __ldcg(n_sel + r);   // written by this warp in this launch: read through L2
+  const int want = i < n ? (int)min((long long)i, kk) + 1 : 0;
+  const int32_t* src = sel + r * stride;
+  const int32_t* ob = o.off + (long long)b * (Nmax + 1);
+  long long keys = 0;
+  for (int q = lane; q < want; q += 32) {
+    const int j = q < cnt ? __ldcg(src + q) : i;
+    o.col_idx[rp + q] = j;
+    keys += ob[j + 1] - ob[j];
+  }
+#pragma unroll
+  for (int s = 16; s > 0; s >>= 1) keys += __shfl_xor_sync(0xffffffffu, keys, s);
+  if (lane == 0) {
+    if (cnt != want) raise_device_flag(o.status, DHSA_DEVFLAG_BAD_SELECTION);
+    o.row_ptr[r] = (int32_t)rp;
+    if (r == (long long)B * Hq * Nmax - 1) o.row_ptr[r + 1] = (int32_t)(rp + want);
+    if (o.cost) o.cost[r] = i < n ? (long long)(ob[i + 1] - ob[i]) * keys : 0;
+  }
+}
+
 __global__ void __launch_bounds__(256) select_kernel(const float* __restrict__ Qp, const float* __restrict__ Kp,
                                                      const float* __restrict__ kn, int Hq, int G, int Nmax,
                                                      const int32_t* __restrict__ n_chunks, int k, int stride,
                                                      long long bh0, long long n_rows,
-                                                     const float* __restrict__ ws, int32_t* __restrict__ sel,
-                                                     int32_t* __restrict__ n_sel) {
+                                                     const float* __restrict__ ws, int32_t* sel, int32_t* n_sel,
+                                                     int B, CsrOut csr) {
   __shared__ int hist_all[8][256];
   const int warp = threadIdx.x >> 5;
   const long long wr = (long long)blockIdx.x * 8 + warp;      // row within the head batch
-  if (wr < n_rows) select_row<false>(Qp, Kp, kn, Hq, G, Nmax, n_chunks, k, stride, bh0, wr, ws, sel, n_sel, hist_all[warp]);
+  if (wr >= n_rows) return;
+  select_row<false>(Qp, Kp, kn, Hq, G, Nmax, n_chunks, k, stride, bh0, wr, ws, sel, n_sel, hist_all[warp]);
+  if (csr.row_ptr) {
+    __syncwarp();
+    csr_row(csr, sel, n_sel, n_chunks, B, Hq, Nmax, stride, bh0 + wr / Nmax, (int)(wr % Nmax));
+  }
 }
 
 // ------------------------------------------------------------------ 3'. row budgets
@@ -537,11 +601,13 @@ long long heads_per_batch(int B, int Hq, int Nmax) {
   return h;
 }
 
+
 // ------------------------------------------------------------------ 4. fused routing
-// Pooling of Q and K, key norms, score tiles and the top-k selection in one
-// cooperative launch, with a grid-wide barrier between the phases that read
-// what the previous one wrote. Each phase runs the same per-warp or
-// per-block code as its separate kernel, so the results are bit-identical.
+// Pooling of Q and K, key norms, score tiles, the top-k selection and (when
+// asked) the block CSR in one cooperative launch, with a grid-wide barrier
+// between the phases that read what the previous one wrote. Each phase runs
+// the same per-warp or per-block code as its separate kernel, so the
+// results are bit-identical.
 struct GridBar {
   unsigned int* count;    // arrivals so far (zeroed before the launch)
   unsigned int* abort;    // set by a block that gave up waiting (zeroed before the launch)
@@ -604,8 +670,8 @@ __global__ void __launch_bounds__(256, 3) route_fused_kernel(const uint4* __rest
                                                           const int32_t* __restrict__ n_chunks, int Nmax, int k,
                                                           int stride, long long hb, float* __restrict__ Qp,
                                                           float* __restrict__ Kp, float* __restrict__ kn,
-                                                          float* __restrict__ scores, int32_t* __restrict__ sel,
-                                                          int32_t* __restrict__ n_sel, GridBar gb) {
+                                                          float* __restrict__ scores, int32_t* sel, int32_t* n_sel,
+                                                          GridBar gb, CsrOut csr) {
   extern __shared__ __align__(16) float sm[];
   const int G = Hq / Hkv;
   const long long gwarp = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
@@ -632,8 +698,13 @@ __global__ void __launch_bounds__(256, 3) route_fused_kernel(const uint4* __rest
       __syncthreads();   // the next tile restages shared memory
     }
     if (!grid_barrier(gb, phase)) return;
-    for (long long wr = gwarp; wr < nh * Nmax; wr += nwarps)
+    for (long long wr = gwarp; wr < nh * Nmax; wr += nwarps) {
       select_row<true>(Qp, Kp, kn, Hq, G, Nmax, n_chunks, k, stride, h0, wr, scores, sel, n_sel, hist);
+      if (csr.row_ptr) {
+        __syncwarp();
+        csr_row(csr, sel, n_sel, n_chunks, B, Hq, Nmax, stride, h0 + wr / Nmax, (int)(wr % Nmax));
+      }
+    }
     if (h0 + hb < total && !grid_barrier(gb, phase)) return;   // the next head batch overwrites the scores
   }
 }
@@ -650,42 +721,41 @@ size_t score_topk_ws_bytes(int B, int Hq, int Nmax) {
 }
 
 int launch_score_topk(const float* Qp, const float* Kp, int B, int Hq, int Hkv, int Nmax, const int32_t* n_chunks,
-                      int k, int32_t* sel, int32_t* n_sel, void* ws, cudaStream_t stream) {
+                      int k, int32_t* sel, int32_t* n_sel, void* ws, const CsrOut& csr, cudaStream_t stream) {
   const int G = Hq / Hkv;
   const int stride = score_topk_stride(k, Nmax);
   float* kn = reinterpret_cast<float*>(static_cast<char*>(ws) + 256);
   const size_t kn_bytes = (sizeof(float) * (size_t)B * Hq * Nmax + 255) & ~size_t(255);
   float* scores = reinterpret_cast<float*>(static_cast<char*>(ws) + 256 + kn_bytes);
-  const long long kv_rows = (long long)B * Hkv * Nmax;
-  key_norm_kernel<<<(unsigned)((kv_rows * 32 + 255) / 256), 256, 0, stream>>>(Kp, kv_rows, kn);
-  int st = launch_status();
-  if (st != DHSA_OK) return st;
   const size_t smem = sizeof(float) * (TR * kHeadDim + TK * kKsStride);
   cudaError_t e = cudaFuncSetAttribute(score_tile_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return cuda_status(e);
+  int st = DHSA_OK;
   const int n_rb = (Nmax + TR - 1) / TR, n_kb = (Nmax + TK - 1) / TK;
   const long long total = (long long)B * Hq, hb = heads_per_batch(B, Hq, Nmax);
   for (long long h0 = 0; h0 < total; h0 += hb) {
     const long long nh = (total - h0 < hb) ? total - h0 : hb;
     dim3 grid((unsigned)(n_rb * n_kb), (unsigned)nh);
-    score_tile_kernel<<<grid, 256, smem, stream>>>(Qp, Kp, Hq, G, Nmax, n_chunks, h0, n_rb, n_kb, scores);
+    // the score tiles also write the key norms the selection reads
+    score_tile_kernel<<<grid, 256, smem, stream>>>(Qp, Kp, Hq, G, Nmax, n_chunks, h0, n_rb, n_kb, scores, kn);
     if ((st = launch_status()) != DHSA_OK) return st;
     const long long rows = nh * Nmax;
     select_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(Qp, Kp, kn, Hq, G, Nmax, n_chunks, k, stride, h0,
-                                                                  rows, scores, sel, n_sel);
+                                                                  rows, scores, sel, n_sel, B, csr);
     if ((st = launch_status()) != DHSA_OK) return st;
   }
   return DHSA_OK;
 }
 
-// All of routing up to the selection in one cooperative launch (workspace as
-// for launch_score_topk; its first 8 bytes hold the grid barrier's counter
-// and abort word). limit_ns bounds each barrier wait; hold_ns > 0 is the test
-// hook that makes block 0 arrive late at the first barrier.
+// All of routing up to the selection (and the CSR when csr.row_ptr is set)
+// in one cooperative launch (workspace as for launch_score_topk; its first 8
+// bytes hold the grid barrier's counter and abort word). limit_ns bounds
+// each barrier wait; hold_ns > 0 is the test hook that makes block 0 arrive
+// late at the first barrier.
 int launch_route_fused(const void* Q, const void* K, int B, int Hq, int Hkv, int L, const int32_t* off,
                        const int32_t* n_chunks, int Nmax, int k, float* Qp, float* Kp, int32_t* sel, int32_t* n_sel,
-                       void* ws, unsigned int* status, unsigned long long limit_ns, unsigned long long hold_ns,
-                       cudaStream_t stream) {
+                       const CsrOut& csr, void* ws, unsigned int* status, unsigned long long limit_ns,
+                       unsigned long long hold_ns, cudaStream_t stream) {
   const int stride = score_topk_stride(k, Nmax);
   float* kn = reinterpret_cast<float*>(static_cast<char*>(ws) + 256);
   const size_t kn_bytes = (sizeof(float) * (size_t)B * Hq * Nmax + 255) & ~size_t(255);
@@ -703,10 +773,11 @@ int launch_route_fused(const void* Q, const void* K, int B, int Hq, int Hkv, int
   GridBar gb{static_cast<unsigned int*>(ws), static_cast<unsigned int*>(ws) + 1, status, limit_ns, hold_ns};
   const uint4* q4 = static_cast<const uint4*>(Q);
   const uint4* k4 = static_cast<const uint4*>(K);
+  CsrOut c = csr;
   void* args[] = {(void*)&q4,     (void*)&k4,   (void*)&B,     (void*)&Hq,   (void*)&Hkv,   (void*)&L,
                   (void*)&off,    (void*)&n_chunks, (void*)&Nmax, (void*)&k, (void*)&stride, (void*)&hb,
                   (void*)&Qp,     (void*)&Kp,   (void*)&kn,    (void*)&scores, (void*)&sel, (void*)&n_sel,
-                  (void*)&gb};
+                  (void*)&gb,     (void*)&c};
   e = cudaLaunchCooperativeKernel((const void*)route_fused_kernel, dim3(per_sm * sms), dim3(256), args, (size_t)smem,
                                   stream);
   return cuda_status(e);
@@ -722,19 +793,16 @@ int launch_score_budget(const float* Qp, const float* Kp, int B, int Hq, int Hkv
   float* kn = reinterpret_cast<float*>(static_cast<char*>(ws) + 256);
   const size_t kn_bytes = (sizeof(float) * (size_t)B * Hq * Nmax + 255) & ~size_t(255);
   float* scores = reinterpret_cast<float*>(static_cast<char*>(ws) + 256 + kn_bytes);
-  const long long kv_rows = (long long)B * Hkv * Nmax;
-  key_norm_kernel<<<(unsigned)((kv_rows * 32 + 255) / 256), 256, 0, stream>>>(Kp, kv_rows, kn);
-  int st = launch_status();
-  if (st != DHSA_OK) return st;
   const size_t smem = sizeof(float) * (TR * kHeadDim + TK * kKsStride);
   cudaError_t e = cudaFuncSetAttribute(score_tile_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return cuda_status(e);
+  int st = DHSA_OK;
   const int n_rb = (Nmax + TR - 1) / TR, n_kb = (Nmax + TK - 1) / TK;
   const long long total = (long long)B * Hq, hb = heads_per_batch(B, Hq, Nmax);
   for (long long h0 = 0; h0 < total; h0 += hb) {
     const long long nh = (total - h0 < hb) ? total - h0 : hb;
     dim3 grid((unsigned)(n_rb * n_kb), (unsigned)nh);
-    score_tile_kernel<<<grid, 256, smem, stream>>>(Qp, Kp, Hq, G, Nmax, n_chunks, h0, n_rb, n_kb, scores);
+    score_tile_kernel<<<grid, 256, smem, stream>>>(Qp, Kp, Hq, G, Nmax, n_chunks, h0, n_rb, n_kb, scores, kn);
     if ((st = launch_status()) != DHSA_OK) return st;
     const long long rows = nh * Nmax;
     budget_select_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(

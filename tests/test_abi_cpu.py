@@ -118,6 +118,25 @@ def test_fused_routing_arguments_rejected_on_host(lib):
     assert f(FAKE, FAKE, 1, 4, 2, 64, 96, FAKE, FAKE, 8, 2, FAKE, FAKE, FAKE, FAKE, FAKE, ws, None) == UNS
     assert f(FAKE, FAKE, 1, 4, 2, 64, 128, FAKE, FAKE, 8, 2, FAKE, FAKE, FAKE, FAKE, None, ws, None) == WS
     assert f(FAKE, FAKE, 1, 4, 2, 64, 128, FAKE, FAKE, 8, 2, FAKE, FAKE, FAKE, FAKE, FAKE, ws - 16, None) == WS
+    g = lib.dhsa_route_topk_csr
+    #          Q     K     B  Hq Hkv  L  hd  off   n_ch Nmax k  Qp    Kp    sel   n_sel rp    ci    cost  ws    bytes
+    assert g(FAKE, FAKE, 1, 4, 2, 64, 128, FAKE, FAKE, 8, 2, FAKE, FAKE, FAKE, FAKE, None, FAKE, None, FAKE, ws,
+             None) == INV
+    assert g(FAKE, FAKE, 1, 4, 2, 64, 128, FAKE, FAKE, 8, 2, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, ws - 16,
+             None) == WS
+
+
+def test_score_topk_csr_arguments_rejected_on_host(lib):
+    INV, WS = 1, 5
+    f = lib.dhsa_chunk_score_topk_csr
+    ws = lib.dhsa_score_topk_workspace_size(1, 4, 8)
+    #          Qp    Kp    B  Hq Hkv Nmax off   n_ch  k  sel   n_sel rp    ci    cost  ws    bytes stream
+    assert f(FAKE, FAKE, 1, 4, 2, 8, None, FAKE, 2, FAKE, FAKE, FAKE, FAKE, None, FAKE, ws, None) == INV
+    assert f(FAKE, FAKE, 1, 4, 2, 8, FAKE, FAKE, 2, FAKE, FAKE, None, FAKE, None, FAKE, ws, None) == INV
+    assert f(FAKE, FAKE, 1, 4, 2, 8, FAKE, FAKE, -1, FAKE, FAKE, FAKE, FAKE, None, FAKE, ws, None) == INV
+    assert f(FAKE, FAKE, 1, 3, 2, 8, FAKE, FAKE, 2, FAKE, FAKE, FAKE, FAKE, None, FAKE, ws, None) == INV
+    assert f(FAKE, FAKE, 1, 4, 2, 8, FAKE, FAKE, 2, FAKE, FAKE, FAKE, FAKE, None, FAKE, ws - 16, None) == WS
+    assert f(FAKE, FAKE, 1, 4, 2, 8, FAKE, FAKE, 2, FAKE, FAKE, FAKE, FAKE, None, None, ws, None) == WS
 
 
 def test_wait_timeout_hook_arguments(lib):

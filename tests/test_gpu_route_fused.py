@@ -1,7 +1,9 @@
-"""The fused routing launch (pooling of Q and K, key norms, score tiles and
-the top-k selection in one cooperative kernel) gives the same pooled vectors,
-selection and CSR as the separate launches, bit for bit; and the layer built
-on it matches the CPU oracle."""
+"""The routing variants agree bit for bit: the separate launches with the
+scan-and-fill CSR build (reference), the selection that writes its CSR rows
+directly (the layer's default under the top-k rule), and the one-launch
+routing (pooling, key norms, score tiles, selection and CSR in one
+cooperative kernel). The layer built on the one-launch routing matches the
+CPU oracle."""
 import numpy as np
 import pytest
 import torch
@@ -30,35 +32,42 @@ CASES = {
     "geometric": I.custom(B=2, Hq=4, Hkv=1, L=3000, lo=1, hi=1024, kind="geometric", mean=40.0, k=6, wid=108),
     "many-chunks": I.custom(B=1, Hq=2, Hkv=1, L=16000, lo=1, hi=3, k=5, wid=120),
     # ~12000 chunks: one head's packed scores (~288 MB) exceed the 256 MiB
-    # score workspace, so the four heads run as four head batches, with a
-    # grid barrier between a batch's selection and the next batch's score
-    # tiles overwriting the same scores
+    # score area, so the four heads run as four head batches, with a barrier
+    # between a batch's selection and the next batch's score tiles
+    # overwriting the same scores (and key norms from the first batch)
     "four-head-batches": I.custom(B=1, Hq=4, Hkv=1, L=24000, lo=1, hi=3, k=5, wid=122),
+    # ~7000 chunks, two heads per batch: the second kv group's norms come
+    # from the second batch's score tiles
+    "two-head-batches": I.custom(B=1, Hq=4, Hkv=2, L=14000, lo=1, hi=3, k=5, wid=123),
+    "ragged-64k": I.WORKLOADS["ragged-64k"],
     "llama8b-32k": I.WORKLOADS["llama8b-32k"],
 }
 
 
 def _layers(lib, d, w):
     t = P.to_dev(d)
-    a = lib.DHSAPrefill(w.B, w.Hq, w.Hkv, w.L, t["off"], t["n_chunks"], w.k)
+    a = lib.DHSAPrefill(w.B, w.Hq, w.Hkv, w.L, t["off"], t["n_chunks"], w.k, csr_from_selection=False)
     f = lib.DHSAPrefill(w.B, w.Hq, w.Hkv, w.L, t["off"], t["n_chunks"], w.k, fused_routing=True)
     return t, a, f
 
 
 @needs_gpu
 @pytest.mark.parametrize("name", list(CASES))
-def test_fused_routing_equals_separate_launches(lib, name):
+def test_routing_variants_agree(lib, name):
     w = CASES[name]
     d = I.make_inputs(w, with_v=False)
     t, a, f = _layers(lib, d, w)
-    a.routing(t["Q"], t["K"])
-    f.routing(t["Q"], t["K"])
+    c = lib.DHSAPrefill(w.B, w.Hq, w.Hkv, w.L, t["off"], t["n_chunks"], w.k)
+    for lay in (a, c, f):
+        lay.col_idx.fill_(-7)
+        lay.routing(t["Q"], t["K"])
     torch.cuda.synchronize()
     assert lib.check_device_status() == 0
-    for x in ("Qp", "Kp", "sel", "n_sel", "row_ptr", "cost"):
-        assert torch.equal(getattr(a, x), getattr(f, x)), x
     nnz = int(a.row_ptr[-1])
-    assert torch.equal(a.col_idx[:nnz], f.col_idx[:nnz])
+    for other in (c, f):
+        for x in ("Qp", "Kp", "sel", "n_sel", "row_ptr", "cost"):
+            assert torch.equal(getattr(a, x), getattr(other, x)), x
+        assert torch.equal(a.col_idx[:nnz], other.col_idx[:nnz])
 
 
 @needs_gpu
