@@ -10,12 +10,15 @@
 // The ranking is decided on the fp64 dot products of the fp32 pooled vectors
 // (fp32 x fp32 products are exact in fp64), but only a handful of scores per
 // row are ever computed in fp64:
-//   1. kn kernel: ||Kp_j||_2 for every pooled key row (rounded up).
-//   2. score kernel: fp32 FFMA scores of 64-row x 128-key tiles of the lower
+//   1. score kernel: fp32 FFMA scores of 64-row x 128-key tiles of the lower
 //      triangle (register-tiled, both operands staged in shared memory),
-//      stored packed per row (row i holds its i scores) in the workspace.
-//   3. select kernel, one warp per row: an 8-bit radix select over the
-//      order-preserving fp32 keys finds the m-th largest fp32 score T. The
+//      stored packed per row (row i holds its i scores) in the workspace;
+//      some of its tiles also write ||Kp_j||_2 of every pooled key row
+//      (rounded up).
+//   2. select kernel, one warp per row (its scores staged once in shared
+//      memory when the row has at most 1024): a radix select in digits of
+//      8 bits over the order-preserving fp32 keys, from the highest bit in
+//      which the row's keys differ, finds the m-th largest fp32 score T. The
 //      fp32 dot product of n = 128 terms is within gamma_n * ||q|| * ||k||
 //      of the exact one (gamma_n = n u / (1 - n u), u = 2^-24), so with D
 //      = 2 gamma_n ||q_i|| max_j ||k_j|| every score above T + D is in the
@@ -200,24 +203,86 @@ __device__ __forceinline__ bool ranks_above(double sa, int ja, double sb, int jb
 // `hist` is that warp's 256-int shared scratch.
 struct Cut {
   double lo, hi, cutE;
+  float lo_f, hi_f;   // the band's bounds rounded inward to fp32: for a float s,
+                      // s >= lo iff s >= lo_f and s <= hi iff s <= hi_f
   int cutJ;
+  int nlist;          // >= 0: the band members inside the cut are the first nlist
+                      // entries of the warp's hist area (no re-scoring needed)
   bool all_band;
 };
 
+constexpr int kRowCap = 1024;   // scores of a row a warp stages in shared memory
+constexpr int kSelectSmem = 8 * kRowCap * (int)sizeof(float);   // dynamic shared memory of the selection kernels
+
+// A row of packed scores: a warp's copy in shared memory when the row fits
+// (every pass of the selection then reads shared memory instead of
+// re-reading global memory with dependent loads), else the row in global
+// memory.
+struct RowSrc {
+  const float* p;
+  bool smem;
+};
+
 template <bool kCoh>
-__device__ Cut topm_cut(const float* __restrict__ row, int c, int m, int* hist, const float* __restrict__ qrow,
+__device__ __forceinline__ float rd(const RowSrc& r, int j) {
+  if constexpr (kCoh) {
+    if (!r.smem) return __ldcg(r.p + j);
+  }
+  return r.p[j];
+}
+
+// one warp: stage row[0 .. c) into its buffer when it fits
+template <bool kCoh>
+__device__ __forceinline__ RowSrc stage_row(const float* row, int c, float* buf) {
+  if (c > kRowCap) return RowSrc{row, false};
+  const int lane = threadIdx.x & 31;
+  for (int j0 = 0; j0 < c; j0 += 256) {
+    float v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int j = j0 + lane + 32 * u;
+      v[u] = j < c ? ldf<kCoh>(row + j) : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int j = j0 + lane + 32 * u;
+      if (j < c) buf[j] = v[u];
+    }
+  }
+  __syncwarp();
+  return RowSrc{buf, true};
+}
+
+template <bool kCoh>
+__device__ Cut topm_cut(const RowSrc& row, int c, int m, int* hist, const float* __restrict__ qrow,
                         const float* __restrict__ Kp, long long kv_row0, const float* __restrict__ kn) {
   const int lane = threadIdx.x & 31;
   const unsigned full = 0xffffffffu;
-  // --- radix select of the m-th largest fp32 key
-  unsigned prefix = 0, mask = 0;
+  // --- radix select of the m-th largest fp32 key, over the bits in which
+  // the row's keys differ: the leading bits all keys share (sign and
+  // exponent, mostly) would put every key in one or two bins and serialise
+  // the histogram's shared-memory atomics
+  unsigned key_hi = 0u, key_lo = 0xffffffffu;
+  for (int j = lane; j < c; j += 32) {
+    const unsigned kk = order_key32(rd<kCoh>(row, j));
+    key_hi = max(key_hi, kk);
+    key_lo = min(key_lo, kk);
+  }
+  key_hi = __reduce_max_sync(full, key_hi);
+  key_lo = __reduce_min_sync(full, key_lo);
+  const unsigned diff = key_hi ^ key_lo;
+  int hi = diff ? 31 - __clz(diff) : -1;      // highest bit still to resolve
+  unsigned mask = diff ? ~((2u << hi) - 1u) : 0xffffffffu;
+  unsigned prefix = key_hi & mask;            // every key equal: the m-th largest is that key
   int need = m;
-  for (int shift = 24; shift >= 0; shift -= 8) {
+  while (hi >= 0) {
+    const int shift = hi >= 7 ? hi - 7 : 0;
+    const unsigned dmask = (2u << (hi - shift)) - 1u;   // a digit of at most 8 bits
     for (int q = lane; q < 256; q += 32) hist[q] = 0;
     __syncwarp();
     for (int j = lane; j < c; j += 32) {
-      const unsigned kk = order_key32(ldf<kCoh>(row + j));
-      if ((kk & mask) == prefix) atomicAdd(&hist[(kk >> shift) & 255], 1);
+      const unsigned kk = order_key32(rd<kCoh>(row, j));
+      if ((kk & mask) == prefix) atomicAdd(&hist[(kk >> shift) & dmask], 1);
     }
     __syncwarp();
     int cq[8], lsum = 0;
@@ -235,7 +300,7 @@ __device__ Cut topm_cut(const float* __restrict__ row, int c, int m, int* hist, 
     const int excl = incl - lsum;
     const unsigned ball = __ballot_sync(full, excl < need && need <= incl);
     const int src = __ffs(ball) - 1;
-    int digit = 0, above = 0;
+    int digit = 0, above = 0, inbin = 0;
     if (lane == src) {
       int run = excl;
 #pragma unroll
@@ -243,6 +308,7 @@ __device__ Cut topm_cut(const float* __restrict__ row, int c, int m, int* hist, 
         if (run + cq[q] >= need) {
           digit = 255 - 8 * lane - q;
           above = run;
+          inbin = cq[q];
           break;
         }
         run += cq[q];
@@ -250,10 +316,44 @@ __device__ Cut topm_cut(const float* __restrict__ row, int c, int m, int* hist, 
     }
     digit = __shfl_sync(full, digit, src);
     above = __shfl_sync(full, above, src);
+    inbin = __shfl_sync(full, inbin, src);
     prefix |= (unsigned)digit << shift;
-    mask |= 0xFFu << shift;
+    mask |= dmask << shift;
     need -= above;
+    hi = shift - 1;
     __syncwarp();
+    if (hi >= 0 && inbin <= 32) {
+      // at most 32 keys share the prefix: gather them (one per lane), sort
+      // them descending and take the need-th; no further histogram passes
+      int base = 0;
+      for (int j0 = 0; j0 < c; j0 += 32) {
+        const int j = j0 + lane;
+        unsigned kk = 0;
+        bool hit = false;
+        if (j < c) {
+          kk = order_key32(rd<kCoh>(row, j));
+          hit = (kk & mask) == prefix;
+        }
+        const unsigned bb = __ballot_sync(full, hit);
+        if (hit) hist[base + __popc(bb & lanemask_lt())] = (int)kk;
+        base += __popc(bb);
+      }
+      __syncwarp();
+      unsigned key = lane < inbin ? (unsigned)hist[lane] : 0u;
+#pragma unroll
+      for (int size = 2; size <= 32; size <<= 1) {
+#pragma unroll
+        for (int stride2 = size >> 1; stride2 > 0; stride2 >>= 1) {
+          const unsigned other = __shfl_xor_sync(full, key, stride2);
+          const bool up = ((lane & size) == 0);        // this block sorts descending
+          const bool lower = ((lane & stride2) == 0);
+          key = (lower == up) ? max(key, other) : min(key, other);
+        }
+      }
+      prefix = __shfl_sync(full, key, need - 1);
+      hi = -1;
+      __syncwarp();
+    }
   }
   const unsigned tu = (prefix & 0x80000000u) ? (prefix & 0x7fffffffu) : ~prefix;
   const double T = (double)__uint_as_float(tu);
@@ -271,39 +371,35 @@ __device__ Cut topm_cut(const float* __restrict__ row, int c, int m, int* hist, 
   Cut cut;
   cut.lo = T - D;
   cut.hi = T + D;
+  cut.lo_f = __double2float_ru(cut.lo);
+  cut.hi_f = __double2float_rd(cut.hi);
   cut.cutE = -INFINITY;
   cut.cutJ = 0x7fffffff;
+  cut.nlist = -1;
+  // one pass: count the scores above the band, and list the band's members
+  // (their first 256 indices, through the free histogram area)
   int a = 0, nc = 0;
-  for (int j = lane; j < c; j += 32) {
-    const double s = (double)ldf<kCoh>(row + j);
-    a += s > cut.hi;
-    nc += (s >= cut.lo && s <= cut.hi);
+  for (int j0 = 0; j0 < c; j0 += 32) {
+    const int j = j0 + lane;
+    bool inb = false, abv = false;
+    if (j < c) {
+      const float s = rd<kCoh>(row, j);
+      abv = s > cut.hi_f;
+      inb = s >= cut.lo_f && s <= cut.hi_f;
+    }
+    const unsigned bb = __ballot_sync(full, inb);
+    const int pos = nc + __popc(bb & lanemask_lt());
+    if (inb && pos < 256) hist[pos] = j;
+    nc += __popc(bb);
+    a += __popc(__ballot_sync(full, abv));
   }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    a += __shfl_xor_sync(full, a, o);
-    nc += __shfl_xor_sync(full, nc, o);
-  }
+  __syncwarp();
   const int r = m - a;              // 1 <= r <= nc
   // --- exact cut (E*, j*) among the band: the r-th by (exact desc, j asc)
   cut.all_band = (r >= nc);
   if (cut.all_band) return cut;
   if (nc <= 32) {
-    // compact the band into lanes 0..nc-1 (through the free histogram area),
-    // score exactly, bitonic sort best-first
-    int base = 0;
-    for (int j0 = 0; j0 < c; j0 += 32) {
-      const int j = j0 + lane;
-      bool inb = false;
-      if (j < c) {
-        const double s = (double)ldf<kCoh>(row + j);
-        inb = s >= cut.lo && s <= cut.hi;
-      }
-      const unsigned bb = __ballot_sync(full, inb);
-      if (inb) hist[base + __popc(bb & lanemask_lt())] = j;
-      base += __popc(bb);
-    }
-    __syncwarp();
+    // the band sits in lanes 0..nc-1: score exactly, bitonic sort best-first
     const int my_j = lane < nc ? hist[lane] : -1;
     __syncwarp();
     double my_e = -INFINITY;
@@ -330,6 +426,10 @@ __device__ Cut topm_cut(const float* __restrict__ row, int c, int m, int* hist, 
     }
     cut.cutE = __shfl_sync(full, my_e, r - 1);
     cut.cutJ = __shfl_sync(full, my_key_j, r - 1);
+    // the r best band members (lanes 0 .. r-1 after the sort), for in_cut
+    if (lane < r) hist[lane] = my_key_j;
+    __syncwarp();
+    cut.nlist = r;
   } else {
     // many candidates (heavy ties): r rounds of "best below the previous pick"
     double pe = INFINITY;
@@ -338,8 +438,8 @@ __device__ Cut topm_cut(const float* __restrict__ row, int c, int m, int* hist, 
       double be = -INFINITY;
       int bj = 0x7fffffff;
       for (int j = lane; j < c; j += 32) {
-        const double s = (double)ldf<kCoh>(row + j);
-        if (s < cut.lo || s > cut.hi) continue;
+        const float s = rd<kCoh>(row, j);
+        if (s < cut.lo_f || s > cut.hi_f) continue;
         const double e = exact_score<kCoh>(qrow, Kp + (kv_row0 + j) * kHeadDim);
         if (ranks_above(pe, pj, e, j) && ranks_above(e, j, be, bj)) {
           be = e;
@@ -365,13 +465,19 @@ __device__ Cut topm_cut(const float* __restrict__ row, int c, int m, int* hist, 
 }
 
 // Is candidate j (fp32 score s) inside the exact top-m described by `cut`?
+// (list: the warp's hist area, holding the cut's band members when listed)
 template <bool kCoh>
 __device__ __forceinline__ bool in_cut(const Cut& cut, float s32, int j, const float* __restrict__ qrow,
-                                       const float* __restrict__ Kp, long long kv_row0) {
-  const double s = (double)s32;
-  if (s > cut.hi) return true;
-  if (s < cut.lo) return false;
-  return cut.all_band || !ranks_above(cut.cutE, cut.cutJ, exact_score<kCoh>(qrow, Kp + (kv_row0 + j) * kHeadDim), j);
+                                       const float* __restrict__ Kp, long long kv_row0, const int* list) {
+  if (s32 > cut.hi_f) return true;
+  if (s32 < cut.lo_f) return false;
+  if (cut.all_band) return true;
+  if (cut.nlist >= 0) {
+    for (int t = 0; t < cut.nlist; ++t)
+      if (list[t] == j) return true;
+    return false;
+  }
+  return !ranks_above(cut.cutE, cut.cutJ, exact_score<kCoh>(qrow, Kp + (kv_row0 + j) * kHeadDim), j);
 }
 
 // one warp: the top-k row wr of the head batch starting at head bh0 (hist:
@@ -381,7 +487,7 @@ __device__ __forceinline__ void select_row(const float* __restrict__ Qp, const f
                                            const float* __restrict__ kn, int Hq, int G, int Nmax,
                                            const int32_t* __restrict__ n_chunks, int k, int stride, long long bh0,
                                            long long wr, const float* __restrict__ ws, int32_t* __restrict__ sel,
-                                           int32_t* __restrict__ n_sel, int* hist) {
+                                           int32_t* __restrict__ n_sel, int* hist, float* rowbuf) {
   const int lane = threadIdx.x & 31;
   const unsigned full = 0xffffffffu;
   const long long bhl = wr / Nmax;
@@ -397,7 +503,7 @@ __device__ __forceinline__ void select_row(const float* __restrict__ Qp, const f
       for (int j = lane; j < i; j += 32) out[j] = j;
       cnt = i;
     } else if (m > 0) {
-      const float* row = ws + bhl * tri(Nmax) + tri(i);
+      const RowSrc row = stage_row<kCoh>(ws + bhl * tri(Nmax) + tri(i), i, rowbuf);
       const long long kv_row0 = ((long long)b * (Hq / G) + hq / G) * Nmax;
       const float* qrow = Qp + (bh * Nmax + i) * kHeadDim;
       const Cut cut = topm_cut<kCoh>(row, i, m, hist, qrow, Kp, kv_row0, kn);
@@ -405,7 +511,7 @@ __device__ __forceinline__ void select_row(const float* __restrict__ Qp, const f
       int written = 0;
       for (int j0 = 0; j0 < i; j0 += 32) {
         const int j = j0 + lane;
-        const bool take = j < i && in_cut<kCoh>(cut, ldf<kCoh>(row + j), j, qrow, Kp, kv_row0);
+        const bool take = j < i && in_cut<kCoh>(cut, rd<kCoh>(row, j), j, qrow, Kp, kv_row0, hist);
         const unsigned bt = __ballot_sync(full, take);
         const int pos = written + __popc(bt & lanemask_lt());
         if (take && pos < m) out[pos] = j;
@@ -475,10 +581,12 @@ __global__ void __launch_bounds__(256) select_kernel(const float* __restrict__ Q
                                                      const float* __restrict__ ws, int32_t* sel, int32_t* n_sel,
                                                      int B, CsrOut csr) {
   __shared__ int hist_all[8][256];
+  extern __shared__ __align__(16) float rowbuf_all[];   // [8][kRowCap]
   const int warp = threadIdx.x >> 5;
   const long long wr = (long long)blockIdx.x * 8 + warp;      // row within the head batch
   if (wr >= n_rows) return;
-  select_row<false>(Qp, Kp, kn, Hq, G, Nmax, n_chunks, k, stride, bh0, wr, ws, sel, n_sel, hist_all[warp]);
+  select_row<false>(Qp, Kp, kn, Hq, G, Nmax, n_chunks, k, stride, bh0, wr, ws, sel, n_sel, hist_all[warp],
+                    rowbuf_all + warp * kRowCap);
   if (csr.row_ptr) {
     __syncwarp();
     csr_row(csr, sel, n_sel, n_chunks, B, Hq, Nmax, stride, bh0 + wr / Nmax, (int)(wr % Nmax));
@@ -504,6 +612,7 @@ __global__ void __launch_bounds__(256) budget_select_kernel(
   __shared__ int mj_all[8][kBudgetCap];      // members, ascending index
   __shared__ double me_all[8][kBudgetCap];   // their exact scores
   __shared__ int ml_all[8][kBudgetCap];      // chunk lengths by rank
+  extern __shared__ __align__(16) float rowbuf_all[];   // [8][kRowCap]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const unsigned full = 0xffffffffu;
   const long long wr = (long long)blockIdx.x * 8 + warp;
@@ -528,7 +637,7 @@ __global__ void __launch_bounds__(256) budget_select_kernel(
     const long long bud = budgets ? (long long)budgets[bh * Nmax + i] : (long long)budget;
     int t = 0;
     if (m > 0 && used0 < bud) {
-      const float* row = ws + bhl * tri(Nmax) + tri(i);
+      const RowSrc row = stage_row<false>(ws + bhl * tri(Nmax) + tri(i), c, rowbuf_all + warp * kRowCap);
       const long long kv_row0 = ((long long)b * (Hq / G) + hq / G) * Nmax;
       const float* qrow = Qp + (bh * Nmax + i) * kHeadDim;
       const bool all = (m == c);
@@ -538,7 +647,7 @@ __global__ void __launch_bounds__(256) budget_select_kernel(
       int nm = 0;
       for (int j0 = 0; j0 < c; j0 += 32) {
         const int j = j0 + lane;
-        const bool take = j < c && (all || in_cut<false>(cut, row[j], j, qrow, Kp, kv_row0));
+        const bool take = j < c && (all || in_cut<false>(cut, rd<false>(row, j), j, qrow, Kp, kv_row0, hist));
         const unsigned bt = __ballot_sync(full, take);
         const int pos = nm + __popc(bt & lanemask_lt());
         if (take && pos < m) mj[pos] = j;
@@ -689,6 +798,7 @@ __global__ void __launch_bounds__(256, 3) route_fused_kernel(const uint4* __rest
   const int n_rb = (Nmax + TR - 1) / TR, n_kb = (Nmax + 32 * kFusedKC - 1) / (32 * kFusedKC);
   const long long total = (long long)B * Hq;
   int* hist = reinterpret_cast<int*>(sm) + (threadIdx.x >> 5) * 256;
+  float* rowbuf = sm + 8 * 256 + (threadIdx.x >> 5) * kRowCap;   // fits in the score tiles' shared memory
   for (long long h0 = 0; h0 < total; h0 += hb) {
     const long long nh = total - h0 < hb ? total - h0 : hb;
     const long long tiles = nh * n_rb * n_kb;
@@ -699,7 +809,7 @@ __global__ void __launch_bounds__(256, 3) route_fused_kernel(const uint4* __rest
     }
     if (!grid_barrier(gb, phase)) return;
     for (long long wr = gwarp; wr < nh * Nmax; wr += nwarps) {
-      select_row<true>(Qp, Kp, kn, Hq, G, Nmax, n_chunks, k, stride, h0, wr, scores, sel, n_sel, hist);
+      select_row<true>(Qp, Kp, kn, Hq, G, Nmax, n_chunks, k, stride, h0, wr, scores, sel, n_sel, hist, rowbuf);
       if (csr.row_ptr) {
         __syncwarp();
         csr_row(csr, sel, n_sel, n_chunks, B, Hq, Nmax, stride, h0 + wr / Nmax, (int)(wr % Nmax));
@@ -729,6 +839,10 @@ int launch_score_topk(const float* Qp, const float* Kp, int B, int Hq, int Hkv, 
   float* scores = reinterpret_cast<float*>(static_cast<char*>(ws) + 256 + kn_bytes);
   const size_t smem = sizeof(float) * (TR * kHeadDim + TK * kKsStride);
   cudaError_t e = cudaFuncSetAttribute(score_tile_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSelectSmem);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(budget_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSelectSmem);
   if (e != cudaSuccess) return cuda_status(e);
   int st = DHSA_OK;
   const int n_rb = (Nmax + TR - 1) / TR, n_kb = (Nmax + TK - 1) / TK;
@@ -740,7 +854,7 @@ int launch_score_topk(const float* Qp, const float* Kp, int B, int Hq, int Hkv, 
     score_tile_kernel<<<grid, 256, smem, stream>>>(Qp, Kp, Hq, G, Nmax, n_chunks, h0, n_rb, n_kb, scores, kn);
     if ((st = launch_status()) != DHSA_OK) return st;
     const long long rows = nh * Nmax;
-    select_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(Qp, Kp, kn, Hq, G, Nmax, n_chunks, k, stride, h0,
+    select_kernel<<<(unsigned)((rows + 7) / 8), 256, kSelectSmem, stream>>>(Qp, Kp, kn, Hq, G, Nmax, n_chunks, k, stride, h0,
                                                                   rows, scores, sel, n_sel, B, csr);
     if ((st = launch_status()) != DHSA_OK) return st;
   }
@@ -795,6 +909,10 @@ int launch_score_budget(const float* Qp, const float* Kp, int B, int Hq, int Hkv
   float* scores = reinterpret_cast<float*>(static_cast<char*>(ws) + 256 + kn_bytes);
   const size_t smem = sizeof(float) * (TR * kHeadDim + TK * kKsStride);
   cudaError_t e = cudaFuncSetAttribute(score_tile_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSelectSmem);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(budget_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSelectSmem);
   if (e != cudaSuccess) return cuda_status(e);
   int st = DHSA_OK;
   const int n_rb = (Nmax + TR - 1) / TR, n_kb = (Nmax + TK - 1) / TK;
@@ -805,7 +923,7 @@ int launch_score_budget(const float* Qp, const float* Kp, int B, int Hq, int Hkv
     score_tile_kernel<<<grid, 256, smem, stream>>>(Qp, Kp, Hq, G, Nmax, n_chunks, h0, n_rb, n_kb, scores, kn);
     if ((st = launch_status()) != DHSA_OK) return st;
     const long long rows = nh * Nmax;
-    budget_select_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(
+    budget_select_kernel<<<(unsigned)((rows + 7) / 8), 256, kSelectSmem, stream>>>(
         Qp, Kp, kn, Hq, G, Nmax, n_chunks, off, budget, budgets, recent, k_max, stride, h0, rows, scores, sel,
         n_sel);
     if ((st = launch_status()) != DHSA_OK) return st;
