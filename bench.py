@@ -24,7 +24,13 @@ import sys
 import threading
 import time
 
-import numpy as np
+# The CPU legs (the oracle) use exactly the host cores this process may run
+# on: BLAS and OpenMP thread pools are sized before numpy loads.
+CORES = len(os.sched_getaffinity(0))
+for _v in ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS", "MKL_NUM_THREADS"):
+    os.environ.setdefault(_v, str(CORES))
+
+import numpy as np  # noqa: E402
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
@@ -35,8 +41,8 @@ ATTN_SRC = os.path.join(ROOT, "long_context_prefill_dhsa_b200", "csrc", "attn_fw
 # launch from an ncu capture of the 32K layer, scaled by tokens (x4) to the
 # 128K layer; only valid for the kernel source it was measured on (the sha256
 # of the kernel's constants and body, see kernel_region_sha).
-ATTN_TRAFFIC = {"sha256_prefix": "d39f1c097e3452e7",
-                "bytes_per_launch": {"llama3.1-8b-32k": 6.417e8, "llama3.1-8b-128k": 2.567e9},
+ATTN_TRAFFIC = {"sha256_prefix": "8326bc3ff5953d82",
+                "bytes_per_launch": {"llama3.1-8b-32k": 6.414e8, "llama3.1-8b-128k": 2.565e9},
                 "source": "ncu --set full capture of the 32K layer; 128K scaled x4 by tokens"}
 PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS = 6650.0, 1590.0
@@ -237,7 +243,7 @@ def cpu_oracle_sample(d, w, seconds, rule=None):
     from oracle import dhsa as ora
     off, nc = d["off"], d["n_chunks"]
     nmax = off.shape[1] - 1
-    cores = len(os.sched_getaffinity(0))
+    cores = int(os.environ.get("OPENBLAS_NUM_THREADS", CORES))
     t0 = time.perf_counter()
     Qp = ora.chunk_pool(ora.bf16_to_f64(d["Q"][:, :1]), off, nc, nmax)
     Kp = ora.chunk_pool(ora.bf16_to_f64(d["K"][:, :1]), off, nc, nmax)

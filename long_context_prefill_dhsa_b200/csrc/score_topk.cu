@@ -181,6 +181,9 @@ __global__ void __launch_bounds__(256, 2) score_tile_kernel(const float* __restr
 template <bool kCoh>
 __device__ double exact_score(const float* __restrict__ q, const float* __restrict__ k) {
   double a0 = 0.0, a1 = 0.0, a2 = 0.0, a3 = 0.0;
+  // unrolled so that the loads of several steps are in flight together (the
+  // rows come from L2; a rolled loop waits for each pair in turn)
+#pragma unroll 8
   for (int d = 0; d < kHeadDim; d += 4) {
     const float4 x = ldf4<kCoh>(q + d);
     const float4 y = ldf4<kCoh>(k + d);
@@ -361,6 +364,7 @@ __device__ Cut topm_cut(const RowSrc& row, int c, int m, int* hist, const float*
   const float4 qv = ldf4<kCoh>(qrow + 4 * lane);
   double qq = (double)qv.x * qv.x + (double)qv.y * qv.y + (double)qv.z * qv.z + (double)qv.w * qv.w;
   float kmax = 0.f;
+#pragma unroll 4
   for (int j = lane; j < c; j += 32) kmax = fmaxf(kmax, ldf<kCoh>(kn + kv_row0 + j));
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
