@@ -189,6 +189,55 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
+// pairs of fp32 in one 64-bit register, for the packed f32x2 operations
+__device__ __forceinline__ uint64_t pk2(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void unpk2(uint64_t v, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
+// 2^x of two values on the FMA pipe, so that the special-function unit is
+// not the only source of the softmax's exponentials. x = j + f with
+// j = round(x), taken by adding 1.5 * 2^23 (the integer lands in the low
+// mantissa bits of the sum) and |f| <= 1/2; 2^f = 1 + f (c1 + f (c2 + f c3)),
+// the coefficients minimising the maximum relative error on [-1/2, 1/2]
+// (exp2_poly.py beside this file fits them; 1.01e-4, twenty times below
+// bf16's rounding step); j is added into the exponent field. x = 0 gives
+// exactly 1; inputs below -125 (masked scores are -inf) give 2^-125.
+constexpr float kExpC1 = 0.69328302f, kExpC2 = 0.24221103f, kExpC3 = 0.05500864f;
+__device__ __forceinline__ void exp2_poly2(uint64_t x2, float& p0, float& p1) {
+  float x0, x1;
+  unpk2(x2, x0, x1);
+  x2 = pk2(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
+  const uint64_t t = add2(x2, pk2(12582912.f, 12582912.f));
+  const uint64_t j = add2(t, pk2(-12582912.f, -12582912.f));
+  const uint64_t f = fma2(j, pk2(-1.f, -1.f), x2);   // exact
+  uint64_t q = fma2(pk2(kExpC3, kExpC3), f, pk2(kExpC2, kExpC2));
+  q = fma2(q, f, pk2(kExpC1, kExpC1));
+  q = fma2(q, f, pk2(1.f, 1.f));
+  float q0, q1, t0, t1;
+  unpk2(q, q0, q1);
+  unpk2(t, t0, t1);
+  p0 = __int_as_float(__float_as_int(q0) + (__float_as_int(t0) << 23));
+  p1 = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
+}
+// one pair of exponentials in this many goes to exp2_poly2 (measured: 1/4 and
+// 1/3 are fastest, 1/2 overloads the FMA pipe, none leaves the MUFU the bound)
+constexpr int kPolyPairEvery = 4;
+
 __device__ __forceinline__ float max3(float a, float b, float c) {
   float r;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
@@ -668,18 +717,29 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_fwd_kernel(const __gr
         if (rescale) m_used = m_new;
         // a row whose keys so far are all masked keeps m = -inf: its p are 0
         const float neg_m = m_used == -INFINITY ? 0.f : -m_used;
-        float rs8[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) rs8[e] = 0.f;
+        // p = 2^(s c - m), two columns per packed operation; the row sum is
+        // kept as four packed partial sums
+        const uint64_t c2 = pk2(c, c), nm2 = pk2(neg_m, neg_m);
+        uint64_t rs2[4] = {0ull, 0ull, 0ull, 0ull};
         uint32_t pk[32];
 #pragma unroll
         for (int cc = 0; cc < 32; ++cc) {
-          const float p0 = fast_exp2(fmaf(__uint_as_float(s[2 * cc]), c, neg_m));
-          const float p1 = fast_exp2(fmaf(__uint_as_float(s[2 * cc + 1]), c, neg_m));
-          rs8[cc & 7] += p0 + p1;
+          const uint64_t x2 = fma2(pk2(__uint_as_float(s[2 * cc]), __uint_as_float(s[2 * cc + 1])), c2, nm2);
+          float p0, p1;
+          if (cc % kPolyPairEvery == kPolyPairEvery - 1) {
+            exp2_poly2(x2, p0, p1);
+          } else {
+            float x0, x1;
+            unpk2(x2, x0, x1);
+            p0 = fast_exp2(x0);
+            p1 = fast_exp2(x1);
+          }
+          rs2[cc & 3] = add2(rs2[cc & 3], pk2(p0, p1));
           pk[cc] = pack_bf16x2(p0, p1);
         }
-        l_sum += ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
+        float r0, r1;
+        unpk2(add2(add2(rs2[0], rs2[1]), add2(rs2[2], rs2[3])), r0, r1);
+        l_sum += r0 + r1;
         // P (bf16 pairs) over the first 32 of this half's 64 S columns
         tmem_st32(tS0 + sb * 128, pk);
         tmem_wait_st();
