@@ -30,9 +30,10 @@
 //   and K (and of the bias blocks), warp 3 = TMA producer of V, warp 1 =
 //   QK^T issuer, warp 14 = PV issuer (one thread each), warp 2 = scheduler
 //   (resolves each work item's chunk list into a shared-memory ring up to 4
-//   items ahead), warps 4-11 = softmax + epilogue: warpgroup 1 takes key
-//   slots 0..63 of every tile and warpgroup 2 slots 64..127, two warps per
-//   TMEM lane quarter (thread = query row = TMEM lane). Warpgroups 0 and 3
+//   items ahead), warps 4-11 = softmax + epilogue: two warps per TMEM lane
+//   quarter, each owning 16 of its 32 query rows with all 128 key slots of a
+//   tile (TMEM shape 16x256b: four threads per row, two rows per thread).
+//   Warpgroups 0 and 3
 //   hand their registers to the softmax warpgroups (setmaxnreg). The two
 //   issuers sit on sub-partitions apart from the K producer: an issuer that
 //   shares one with the K producer measurably slows that sub-partition's
@@ -48,17 +49,21 @@
 //   With two issuing threads the tensor pipe keeps work queued while either
 //   one waits on a barrier.
 // * TMEM (512 columns): three S buffers (3 x 128 fp32 columns) and the O
-//   accumulator (128 columns). P (bf16) is written back into the S buffer it
-//   came from, each warp into its own half, and consumed from TMEM by the PV
-//   MMA (A in TMEM, V as an N-major shared-memory operand). The QK^T issuer
-//   runs up to three tiles ahead of the PV.
-// * Online softmax in the log2 domain. The two warps of a lane quarter trade
-//   their half-row maxima through shared memory once per tile, then each
-//   exponentiates its 64 columns and keeps its own partial row sum (the two
-//   are added in the epilogue). The running max is only raised (and O
-//   rescaled in TMEM, each warp its half of the columns) when it grows by
-//   more than 8 (a factor 256), which keeps O / l exact while skipping nearly
-//   all rescales; only then does the softmax wait for the previous PV.
+//   accumulator (128 columns). P (bf16 pairs) is written back into the first
+//   64 columns of the S buffer it came from (shape 16x128b, where each
+//   thread's packed pairs land on their own lane and column) and consumed
+//   from TMEM by the PV MMA (A in TMEM, V as an N-major shared-memory
+//   operand). The QK^T issuer runs up to three tiles ahead of the PV.
+// * Online softmax in the log2 domain. A row's maximum is the max of its four
+//   threads' 32 columns, combined with two shuffles: the two warps of a lane
+//   quarter trade nothing per tile. One exponential pair in four is computed
+//   on the FMA pipe (exp2_poly2), the rest by the MUFU; the scale and the
+//   row sums use packed f32x2 operations. The running max is only raised (and
+//   O rescaled in TMEM, each warp its own rows) when it grows by more than 8
+//   (a factor 256), which keeps O / l exact while skipping nearly all
+//   rescales; only then does the softmax wait for the previous PV. At the
+//   end of an item the row sums go through shared memory to the epilogue's
+//   32x32b layout, where each warp writes 64 output columns of 32 rows.
 // * Every mbarrier wait is bounded; a timeout sets DHSA_DEVFLAG_WAIT_TIMEOUT,
 //   the CTA drains its own in-flight copies and MMAs (again bounded), frees
 //   its TMEM and exits.
@@ -136,8 +141,8 @@ constexpr uint32_t OFF_ONES = OFF_V + NSV * kTileBytes;         // 4 KB
 constexpr uint32_t OFF_BIAS = OFF_ONES + kBiasBytes;            // NSK x 4 KB
 constexpr uint32_t OFF_TINFO = OFF_BIAS + NSK * kBiasBytes;    // NTOK int4 tile descriptors
 constexpr uint32_t OFF_SLOT = OFF_TINFO + NTOK * 16;
-constexpr uint32_t OFF_XCHG = OFF_SLOT + NSLOT * sizeof(ItemSlot);   // 2 x 2 x 128 floats, twice
-constexpr uint32_t OFF_BAR = OFF_XCHG + 2 * 2 * 2 * BM * 4;
+constexpr uint32_t OFF_XCHG = OFF_SLOT + NSLOT * sizeof(ItemSlot);   // row sums, [item parity][row]
+constexpr uint32_t OFF_BAR = OFF_XCHG + 2 * BM * 4;
 enum {
   B_QFULL = 0,
   B_QEMPTY = B_QFULL + 2,
@@ -153,8 +158,7 @@ enum {
   B_OFINAL = B_PVDONE + NSB,
   B_FINAL = B_OFINAL + 1,
   B_FINALPV = B_FINAL + 1,
-  B_XMAX = B_FINALPV + 1,        // [quarter][tile parity]: the softmax pair's row-max exchange
-  B_XSUM = B_XMAX + 8,           // [quarter][item parity]: the pair's row-sum exchange
+  B_XSUM = B_FINALPV + 1,        // [quarter][item parity]: the softmax pair's row-sum hand-over
   B_TEARDOWN = B_XSUM + 8,
   B_COUNT = B_TEARDOWN + 1
 };
@@ -216,12 +220,15 @@ __device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
 // the coefficients minimising the maximum relative error on [-1/2, 1/2]
 // (exp2_poly.py beside this file fits them; 1.01e-4, twenty times below
 // bf16's rounding step); j is added into the exponent field. x = 0 gives
-// exactly 1; inputs below -125 (masked scores are -inf) give 2^-125.
+// exactly 1. Inputs are clamped at -127, where j = -127 and f = 0 make the
+// sum's bits exactly +0: masked scores (-inf) give P = 0 as the MUFU does.
+// On (-127, -126) the result lies in [0, 2^-126); for j = -127, f >= 0, so
+// the exponent field never borrows into the sign.
 constexpr float kExpC1 = 0.69328302f, kExpC2 = 0.24221103f, kExpC3 = 0.05500864f;
 __device__ __forceinline__ void exp2_poly2(uint64_t x2, float& p0, float& p1) {
   float x0, x1;
   unpk2(x2, x0, x1);
-  x2 = pk2(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
+  x2 = pk2(fmaxf(x0, -127.f), fmaxf(x1, -127.f));
   const uint64_t t = add2(x2, pk2(12582912.f, 12582912.f));
   const uint64_t j = add2(t, pk2(-12582912.f, -12582912.f));
   const uint64_t f = fma2(j, pk2(-1.f, -1.f), x2);   // exact
@@ -242,19 +249,6 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
   float r;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
   return r;
-}
-
-// maximum of 64 scores: 8 independent chains of three-input max
-__device__ __forceinline__ float max64(const uint32_t (&s)[64]) {
-  float m[8];
-#pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    m[e] = max3(__uint_as_float(s[e]), __uint_as_float(s[e + 8]), __uint_as_float(s[e + 16]));
-    m[e] = max3(m[e], __uint_as_float(s[e + 24]), __uint_as_float(s[e + 32]));
-    m[e] = max3(m[e], __uint_as_float(s[e + 40]), __uint_as_float(s[e + 48]));
-    m[e] = fmaxf(m[e], __uint_as_float(s[e + 56]));
-  }
-  return max3(max3(m[0], m[1], m[2]), max3(m[3], m[4], m[5]), fmaxf(m[6], m[7]));
 }
 
 // byte offset of element (row, k) in a 128 x 16 bf16 K-major block without swizzle
@@ -322,10 +316,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_fwd_kernel(const __gr
       mbar_init(bar(B_OFINAL), 1);
       mbar_init(bar(B_FINAL), 1);
       mbar_init(bar(B_FINALPV), 1);
-      for (int s = 0; s < 8; ++s) {
-        mbar_init(bar(B_XMAX + s), 2);
-        mbar_init(bar(B_XSUM + s), 2);
-      }
+      for (int s = 0; s < 8; ++s) mbar_init(bar(B_XSUM + s), 2);
       mbar_init(bar(B_TEARDOWN), kThreads / 32 - 1);
       fence_mbar_init();
       prefetch_tmap(&maps.q);
@@ -622,8 +613,8 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_fwd_kernel(const __gr
 #pragma unroll
           for (int ks = 0; ks < BN / 16; ++ks) {
             const uint64_t bdesc = smem_desc_sw128(v0 + ks * 2048, kHalfBytes, 1024);
-            // P of key slots 0..63 sits in S columns 0..31, of slots 64..127 in 64..95
-            mma_ts(tO, tS0 + sb * 128 + (ks >> 2) * 64 + (ks & 3) * 8, bdesc, idesc_pv,
+            // P of key slots 16ks .. 16ks + 15 sits in S columns 8ks .. 8ks + 7
+            mma_ts(tO, tS0 + sb * 128 + ks * 8, bdesc, idesc_pv,
                    (kt > 0 || ks > 0) ? 1u : 0u);
           }
           mma_commit(bar(B_PVDONE + sb));
@@ -637,20 +628,24 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_fwd_kernel(const __gr
     }
   } else if (warp >= W_SOFTMAX0 && warp < W_SOFTMAX0 + 8) {
     // ============================================================ softmax + epilogue
-    // Two warps per TMEM lane quarter: warpgroup 1 takes key slots 0..63 of
-    // every tile, warpgroup 2 slots 64..127 (so each SM sub-partition runs two
-    // softmax warps). The pair agrees on the row max through shared memory
-    // once per tile; each keeps its own partial row sum and rescales and
-    // writes its own half of the O columns.
+    // Two warps per TMEM lane quarter, each owning 16 of its 32 query rows
+    // with all 128 key slots of every tile. TMEM shape 16x256b: thread t holds
+    // rows t/4 and t/4 + 8 of the warp's 16, 32 columns of each; the four
+    // threads of a row combine their maxima with two shuffles, so the warps
+    // trade nothing per tile and need not run in step.
     const int quarter = warp & 3;             // TMEM lanes 32*quarter .. +31
     const int half = (warp - W_SOFTMAX0) >> 2;
     regs_inc<kRegsSoftmax>();
-    const int row = quarter * 32 + lane;      // query row within the tile
-    const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
-    const uint32_t tS0 = tmem + lane_addr + half * 64, tO = tmem + lane_addr + 384 + half * 64;
-    float* xmax = reinterpret_cast<float*>(smem + OFF_XCHG);    // [buffer][half][row]
-    float* xsum = xmax + 2 * 2 * BM;                             // [buffer][half][row]
+    const int cq = lane & 3;
+    const int rowA = quarter * 32 + half * 16 + (lane >> 2), rowB = rowA + 8;   // query rows within the tile
+    const uint32_t tS0 = tmem + ((uint32_t)(quarter * 32 + half * 16) << 16);
+    const uint32_t tO16 = tS0 + 384;
+    // epilogue: 32x32b, thread = row quarter*32 + lane, O columns half*64 .. +63
+    const int row = quarter * 32 + lane;
+    const uint32_t tO = tmem + ((uint32_t)(quarter * 32) << 16) + 384 + half * 64;
+    float* xsum = reinterpret_cast<float*>(smem + OFF_XCHG);    // [item parity][row]
     const float c = p.scale_log2;
+    const uint64_t c2 = pk2(c, c);
     uint32_t g = 0;
     int n_local = 0;
     for (;; ++n_local) {
@@ -660,105 +655,154 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_fwd_kernel(const __gr
       if (M.T < 0) break;                  // end of the work list
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(B_SLEMPTY + sl));
-      const int qt = M.q0 + row;
-      float m_used = -INFINITY, l_sum = 0.f;
+      const int qtA = M.q0 + rowA, qtB = M.q0 + rowB;
+      float mA = -INFINITY, mB = -INFINITY, lA = 0.f, lB = 0.f;
       bool ok = true;
       for (int kt = 0; kt < M.T; ++kt, ++g) {
-        const int sb = g % NSB, tk = g % NTOK, xb = g & 1;
-        if (!fl.wait(bar(B_SFULL + sb), (g / NSB) & 1) || !fl.wait(bar(B_TOKFULL + tk), (g / NTOK) & 1)) {
+        const int sb = g % NSB, tk = g % NTOK;
+        // both barriers tested back to back (the usual case: both complete)
+        const bool s_done = mbar_test_wait(bar(B_SFULL + sb), (g / NSB) & 1);
+        const bool t_done = mbar_test_wait(bar(B_TOKFULL + tk), (g / NTOK) & 1);
+        if (!(s_done && t_done) &&
+            (!fl.wait(bar(B_SFULL + sb), (g / NSB) & 1) || !fl.wait(bar(B_TOKFULL + tk), (g / NTOK) & 1))) {
           ok = false;
           break;
         }
         tc_fence_after();
+        // s[4j + e]: row A, column 8j + 2cq + e; s[4j + 2 + e]: row B, same column
         uint32_t s[64];
-        tmem_ld32(tS0 + sb * 128 + 0, *reinterpret_cast<uint32_t(*)[32]>(s + 0));
-        tmem_ld32(tS0 + sb * 128 + 32, *reinterpret_cast<uint32_t(*)[32]>(s + 32));
+        tmem_ld_16x256b_x8(tS0 + sb * 128 + 0, *reinterpret_cast<uint32_t(*)[32]>(s + 0));
+        tmem_ld_16x256b_x8(tS0 + sb * 128 + 64, *reinterpret_cast<uint32_t(*)[32]>(s + 32));
         tmem_wait_ld();
         const int4 ti = tile_info[tk];
         if (ti.x) {
-          // keys after query token qt: the slots from thr on (slots past the
-          // diagonal piece are padding and already -inf)
-          const int thr = max(qt + ti.z + 1, ti.y) - half * 64;
+          // keys after the query token: the slots from the row's threshold on
+          const int thrA = max(qtA + ti.z + 1, ti.y), thrB = max(qtB + ti.z + 1, ti.y);
 #pragma unroll
-          for (int e = 0; e < 64; ++e)
-            if (e >= thr) s[e] = __float_as_uint(-INFINITY);
+          for (int j = 0; j < 16; ++j)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const int col = 8 * j + 2 * cq + e;
+              if (col >= thrA) s[4 * j + e] = __float_as_uint(-INFINITY);
+              if (col >= thrB) s[4 * j + 2 + e] = __float_as_uint(-INFINITY);
+            }
         }
-        float mx = max64(s);
-        // exchange the half-row maxima with the partner warp (same rows)
-        xmax[(xb * 2 + half) * BM + row] = mx;
-        tc_fence_before();
         __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(bar(B_TOKEMPTY + tk));
-          mbar_arrive(bar(B_XMAX + quarter * 2 + xb));
+        if (lane == 0) mbar_arrive(bar(B_TOKEMPTY + tk));
+        // row maxima: two chains per row over the thread's 32 columns
+        auto S = [&](int e) { return __uint_as_float(s[e]); };
+        float a0 = fmaxf(S(0), S(1)), a1 = fmaxf(S(4), S(5));
+        float b0 = fmaxf(S(2), S(3)), b1 = fmaxf(S(6), S(7));
+#pragma unroll
+        for (int j = 2; j < 16; j += 2) {
+          a0 = max3(a0, S(4 * j), S(4 * j + 1));
+          a1 = max3(a1, S(4 * j + 4), S(4 * j + 5));
+          b0 = max3(b0, S(4 * j + 2), S(4 * j + 3));
+          b1 = max3(b1, S(4 * j + 6), S(4 * j + 7));
         }
-        if (!fl.wait(bar(B_XMAX + quarter * 2 + xb), (g >> 1) & 1)) { ok = false; break; }
-        tc_fence_after();
-        mx = fmaxf(mx, xmax[(xb * 2 + (half ^ 1)) * BM + row]);
-        const float m_new = fmaxf(m_used, mx * c);
-        const bool rescale = m_new > m_used + 8.0f;  // also true on the first tile
-        if (kt > 0 && __any_sync(0xffffffffu, rescale)) {
+        float xA = fmaxf(a0, a1), xB = fmaxf(b0, b1);
+        xA = fmaxf(xA, __shfl_xor_sync(0xffffffffu, xA, 1));
+        xB = fmaxf(xB, __shfl_xor_sync(0xffffffffu, xB, 1));
+        xA = fmaxf(xA, __shfl_xor_sync(0xffffffffu, xA, 2));
+        xB = fmaxf(xB, __shfl_xor_sync(0xffffffffu, xB, 2));
+        const float nA = fmaxf(mA, xA * c), nB = fmaxf(mB, xB * c);
+        const bool rA = nA > mA + 8.0f, rB = nB > mB + 8.0f;   // also true on the first tile
+        if (kt > 0 && __any_sync(0xffffffffu, rA || rB)) {
           // O may only be touched once the previous tile's PV has finished
           if (!fl.wait(bar(B_PVDONE + (g - 1) % NSB), ((g - 1) / NSB) & 1)) { ok = false; break; }
           tc_fence_after();
-          const float f = rescale ? fast_exp2(m_used - m_new) : 1.f;
+          const float fA = rA ? fast_exp2(mA - nA) : 1.f, fB = rB ? fast_exp2(mB - nB) : 1.f;
 #pragma unroll
-          for (int c4 = 0; c4 < 2; ++c4) {
-            uint32_t o[32];
-            tmem_ld32(tO + 32 * c4, o);
+          for (int c4 = 0; c4 < 4; ++c4) {
+            uint32_t o[16];
+            tmem_ld_16x256b_x4(tO16 + 32 * c4, o);
             tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
-            tmem_st32(tO + 32 * c4, o);
+            for (int j = 0; j < 4; ++j) {
+              o[4 * j + 0] = __float_as_uint(__uint_as_float(o[4 * j + 0]) * fA);
+              o[4 * j + 1] = __float_as_uint(__uint_as_float(o[4 * j + 1]) * fA);
+              o[4 * j + 2] = __float_as_uint(__uint_as_float(o[4 * j + 2]) * fB);
+              o[4 * j + 3] = __float_as_uint(__uint_as_float(o[4 * j + 3]) * fB);
+            }
+            tmem_st_16x256b_x4(tO16 + 32 * c4, o);
           }
           tmem_wait_st();
-          if (rescale) l_sum *= f;
+          if (rA) lA *= fA;
+          if (rB) lB *= fB;
         }
-        if (rescale) m_used = m_new;
+        if (rA) mA = nA;
+        if (rB) mB = nB;
         // a row whose keys so far are all masked keeps m = -inf: its p are 0
-        const float neg_m = m_used == -INFINITY ? 0.f : -m_used;
-        // p = 2^(s c - m), two columns per packed operation; the row sum is
-        // kept as four packed partial sums
-        const uint64_t c2 = pk2(c, c), nm2 = pk2(neg_m, neg_m);
-        uint64_t rs2[4] = {0ull, 0ull, 0ull, 0ull};
-        uint32_t pk[32];
+        const uint64_t nA2 = pk2(mA == -INFINITY ? 0.f : -mA, mA == -INFINITY ? 0.f : -mA);
+        const uint64_t nB2 = pk2(mB == -INFINITY ? 0.f : -mB, mB == -INFINITY ? 0.f : -mB);
+        uint64_t rsA[2] = {0ull, 0ull}, rsB[2] = {0ull, 0ull};
+        // two halves of 8 column groups; pk[2u]: P of row A, key slots
+        // 16j + 4cq + {0..3} (j = 8h + u) packed as bf16 pairs at column
+        // 4j + cq (16x128b: thread t writes lane t/4 from pk[2u] and lane
+        // t/4 + 8 from pk[2u + 1])
 #pragma unroll
-        for (int cc = 0; cc < 32; ++cc) {
-          const uint64_t x2 = fma2(pk2(__uint_as_float(s[2 * cc]), __uint_as_float(s[2 * cc + 1])), c2, nm2);
-          float p0, p1;
-          if (cc % kPolyPairEvery == kPolyPairEvery - 1) {
-            exp2_poly2(x2, p0, p1);
-          } else {
-            float x0, x1;
-            unpk2(x2, x0, x1);
-            p0 = fast_exp2(x0);
-            p1 = fast_exp2(x1);
+        for (int h = 0; h < 2; ++h) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const int j = 8 * h + u;
+            const uint64_t xa = fma2(pk2(__uint_as_float(s[4 * j]), __uint_as_float(s[4 * j + 1])), c2, nA2);
+            const uint64_t xb = fma2(pk2(__uint_as_float(s[4 * j + 2]), __uint_as_float(s[4 * j + 3])), c2, nB2);
+            float a0, a1, b0, b1;
+            if (j % kPolyPairEvery == kPolyPairEvery - 1) {
+              exp2_poly2(xa, a0, a1);
+              exp2_poly2(xb, b0, b1);
+            } else {
+              float x0, x1;
+              unpk2(xa, x0, x1);
+              a0 = fast_exp2(x0);
+              a1 = fast_exp2(x1);
+              unpk2(xb, x0, x1);
+              b0 = fast_exp2(x0);
+              b1 = fast_exp2(x1);
+            }
+            rsA[u & 1] = add2(rsA[u & 1], pk2(a0, a1));
+            rsB[u & 1] = add2(rsB[u & 1], pk2(b0, b1));
+            pk[2 * u] = pack_bf16x2(a0, a1);
+            pk[2 * u + 1] = pack_bf16x2(b0, b1);
           }
-          rs2[cc & 3] = add2(rs2[cc & 3], pk2(p0, p1));
-          pk[cc] = pack_bf16x2(p0, p1);
+          // P (bf16 pairs) over S columns 32h .. 32h + 31
+          tmem_st_16x128b_x8(tS0 + sb * 128 + 32 * h, pk);
         }
-        float r0, r1;
-        unpk2(add2(add2(rs2[0], rs2[1]), add2(rs2[2], rs2[3])), r0, r1);
-        l_sum += r0 + r1;
-        // P (bf16 pairs) over the first 32 of this half's 64 S columns
-        tmem_st32(tS0 + sb * 128, pk);
+        {
+          float r0, r1;
+          unpk2(add2(rsA[0], rsA[1]), r0, r1);
+          lA += r0 + r1;
+          unpk2(add2(rsB[0], rsB[1]), r0, r1);
+          lB += r0 + r1;
+        }
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(B_PREADY + sb));
       }
       if (!ok) break;
-      // epilogue: O / l -> bf16 over this warp's 64 columns (an empty key
-      // set, which valid CSR input never has, writes zeros)
+      // epilogue: the row sums (four threads per row) go through shared
+      // memory to the 32x32b layout; O / l -> bf16, each warp 64 columns of
+      // the quarter's 32 rows (an empty key set, which valid CSR input never
+      // has, writes zeros)
+      lA += __shfl_xor_sync(0xffffffffu, lA, 1);
+      lB += __shfl_xor_sync(0xffffffffu, lB, 1);
+      lA += __shfl_xor_sync(0xffffffffu, lA, 2);
+      lB += __shfl_xor_sync(0xffffffffu, lB, 2);
       const int lb = n_local & 1;
-      xsum[(lb * 2 + half) * BM + row] = l_sum;
+      if (cq == 0) {
+        xsum[lb * BM + rowA] = lA;
+        xsum[lb * BM + rowB] = lB;
+      }
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(B_XSUM + quarter * 2 + lb));
       if (!fl.wait(bar(B_XSUM + quarter * 2 + lb), (n_local >> 1) & 1)) break;
-      const float l_tot = l_sum + xsum[(lb * 2 + (half ^ 1)) * BM + row];
+      const float l_tot = xsum[lb * BM + row];
       if (!fl.wait(bar(B_OFINAL), n_local & 1)) break;
       tc_fence_after();
       const float inv_l = M.T > 0 ? 1.f / l_tot : 0.f;
+      const int qt = M.q0 + row;
       __nv_bfloat16* orow = p.O + ((long long)M.q_row0 + qt) * kHeadDim + half * 64;
 #pragma unroll
       for (int c4 = 0; c4 < 2; ++c4) {

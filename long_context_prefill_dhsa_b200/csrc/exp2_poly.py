@@ -12,7 +12,8 @@ maximum) gives exactly 1. c1..c3 minimise the maximum relative error
 
 Run `python exp2_poly.py` to print the coefficients, rounded to fp32, and the
 relative error of the fp32 evaluation (magic-constant rounding, FMA Horner
-steps, exponent add) over the softmax's input range [-125, 8].
+steps, exponent add) over [-126, 8]; below -126 the kernel's clamp at -127
+gives values in [0, 2^-126), exactly 0 from -127 down.
 """
 import numpy as np
 from scipy.optimize import linprog
@@ -43,7 +44,7 @@ def _fma32(a, b, d):
 
 def exp2_fp32(x, c):
     """The kernel's fp32 steps, each rounded to fp32."""
-    x = np.maximum(np.asarray(x, np.float32), np.float32(-125.0))
+    x = np.maximum(np.asarray(x, np.float32), np.float32(-127.0))
     t = (x + np.float32(12582912.0)).astype(np.float32)   # 1.5 * 2^23
     j = (t - np.float32(12582912.0)).astype(np.float32)
     fr = (x.astype(np.float64) - j.astype(np.float64)).astype(np.float32)
@@ -59,9 +60,9 @@ def main():
     print("c1, c2, c3 =", ", ".join(f"{v:.8f}f" for v in c))
     print(f"minimax relative error of the polynomial: {e:.3e}")
     rng = np.random.default_rng(0)
-    x = np.concatenate([rng.uniform(-125, 8, 1_000_000), np.linspace(-3, 3, 100_001)]).astype(np.float32)
+    x = np.concatenate([rng.uniform(-126, 8, 1_000_000), np.linspace(-3, 3, 100_001)]).astype(np.float32)
     rel = np.abs(exp2_fp32(x, c) / np.exp2(x.astype(np.float64)) - 1.0)
-    print(f"fp32 evaluation over [-125, 8]: max relative error {rel.max():.3e}")
+    print(f"fp32 evaluation over [-126, 8]: max relative error {rel.max():.3e}")
 
 
 if __name__ == "__main__":

@@ -36,16 +36,16 @@ def test_fp32_steps_within_the_bound():
     g = _gen()
     c = _kernel_coeffs()
     rng = np.random.default_rng(1)
-    x = np.concatenate([rng.uniform(-125, 8, 400_000), np.linspace(-1.5, 1.5, 30_001),
-                        np.arange(-125, 9) + 0.5, np.arange(-124, 9) - 0.49999997]).astype(np.float32)
-    assert x.min() >= -125.0   # below that the kernel clamps (checked separately)
+    x = np.concatenate([rng.uniform(-126, 8, 400_000), np.linspace(-1.5, 1.5, 30_001),
+                        np.arange(-126, 9) + 0.5, np.arange(-125, 9) - 0.49999997]).astype(np.float32)
+    assert x.min() >= -126.0   # below that the results are only bounded (checked separately)
     rel = np.abs(g.exp2_fp32(x, c).astype(np.float64) / np.exp2(x.astype(np.float64)) - 1.0)
     assert rel.max() < 1.05e-4
 
 
 def test_integers_are_exact_powers_of_two():
     # f = 0 there, the polynomial is exactly 1 and only the exponent add acts
-    j = np.arange(-125, 9)
+    j = np.arange(-126, 9)
     v = _gen().exp2_fp32(j.astype(np.float32), _kernel_coeffs())
     assert [float(a) for a in v] == [math.ldexp(1.0, int(e)) for e in j]
 
@@ -53,8 +53,12 @@ def test_integers_are_exact_powers_of_two():
 def test_masked_and_halfway_inputs():
     g = _gen()
     c = _kernel_coeffs()
-    lo = g.exp2_fp32(np.array([-np.inf, -1e30, -126.0], np.float32), c)
-    assert np.all(lo > 0) and np.all(lo <= 2.0 ** -124)
+    # masked scores are -inf: P must be exactly 0, as the MUFU's 2^-inf is
+    lo = g.exp2_fp32(np.array([-np.inf, -1e30, -200.0, -127.0], np.float32), c)
+    assert [float(v) for v in lo] == [0.0, 0.0, 0.0, 0.0]
+    # between -127 and -126 only a bound holds: non-negative, below 2^-126
+    mid = g.exp2_fp32(np.linspace(-127, -126, 100_001).astype(np.float32), c)
+    assert np.all(mid >= 0) and np.all(mid <= 2.0 ** -126) and np.all(np.isfinite(mid))
     # x = -0.5 and +0.5 sit at the ends of the fitted interval
     v = g.exp2_fp32(np.array([-0.5, 0.5], np.float32), c).astype(np.float64)
     assert np.all(np.abs(v / np.exp2([-0.5, 0.5]) - 1) < 1.05e-4)
