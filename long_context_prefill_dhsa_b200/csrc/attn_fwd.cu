@@ -33,6 +33,11 @@
 //   items ahead), warps 4-11 = softmax + epilogue: two warps per TMEM lane
 //   quarter, each owning 16 of its 32 query rows with all 128 key slots of a
 //   tile (TMEM shape 16x256b: four threads per row, two rows per thread).
+//   Tile row r sits in TMEM lane 32 (r mod 4) + r / 4 (Q is loaded through
+//   four views of every fourth row), so the valid rows of a partly filled
+//   tile spread over all four lane quarters; a warp whose 16 rows are all
+//   past the chunk's end only keeps the barrier counts, and its
+//   sub-partition's other warp runs alone.
 //   Warpgroups 0 and 3
 //   hand their registers to the softmax warpgroups (setmaxnreg). The two
 //   issuers sit on sub-partitions apart from the K producer: an issuer that
@@ -94,7 +99,7 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint16_t kBf16One = 0x3F80, kBf16NegInf = 0xFF80;
 
 struct AttnMaps {
-  CUtensorMap q;      // box 64 x 128 rows
+  CUtensorMap q[4];   // rows r, r+4, r+8, ... of Q (r = 0..3), box 64 x 32 rows
   CUtensorMap k[16];  // boxes 64 cols x 8*(n+1) rows: one TMA per chunk piece and head-dim half
   CUtensorMap v[16];
 };
@@ -319,7 +324,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_fwd_kernel(const __gr
       for (int s = 0; s < 8; ++s) mbar_init(bar(B_XSUM + s), 2);
       mbar_init(bar(B_TEARDOWN), kThreads / 32 - 1);
       fence_mbar_init();
-      prefetch_tmap(&maps.q);
+      for (int r = 0; r < 4; ++r) prefetch_tmap(&maps.q[r]);
       for (int s = 0; s < 16; ++s) {
         prefetch_tmap(&maps.k[s]);
         prefetch_tmap(&maps.v[s]);
@@ -423,11 +428,16 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_fwd_kernel(const __gr
       const int ms = n_local & 1;
       if (kprod) {
         if (n_local >= 2 && !fl.wait(bar(B_QEMPTY + ms), ((n_local >> 1) - 1) & 1)) break;
-        if (lane == 0) {
-          mbar_arrive_expect_tx(bar(B_QFULL + ms), kTileBytes);
-          const uint32_t dq = sbase + OFF_Q + ms * kTileBytes;
-          tma_load_2d(dq, &maps.q, bar(B_QFULL + ms), 0, M.q_row0 + M.q0);
-          tma_load_2d(dq + kHalfBytes, &maps.q, bar(B_QFULL + ms), 64, M.q_row0 + M.q0);
+        // tile row r goes to TMEM lane 32 (r mod 4) + r / 4: lane q loads
+        // rows q, q + 4, ..., q + 124 into the 32 rows of lane quarter q
+        if (lane == 0) mbar_arrive_expect_tx(bar(B_QFULL + ms), kTileBytes);
+        __syncwarp();
+        if (lane < 4) {
+          const long long G = (long long)M.q_row0 + M.q0 + lane;
+          const CUtensorMap* mq = &maps.q[G & 3];
+          const uint32_t dq = sbase + OFF_Q + ms * kTileBytes + lane * 4096;
+          tma_load_2d(dq, mq, bar(B_QFULL + ms), 0, (int)(G >> 2));
+          tma_load_2d(dq + kHalfBytes, mq, bar(B_QFULL + ms), 64, (int)(G >> 2));
         }
       }
       const int32_t* ob = p.off + (long long)M.b * (p.Nmax + 1);
@@ -637,11 +647,14 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_fwd_kernel(const __gr
     const int half = (warp - W_SOFTMAX0) >> 2;
     regs_inc<kRegsSoftmax>();
     const int cq = lane & 3;
-    const int rowA = quarter * 32 + half * 16 + (lane >> 2), rowB = rowA + 8;   // query rows within the tile
+    // TMEM lane 32q + l holds query row 4l + q of the tile
+    const int tlA = quarter * 32 + half * 16 + (lane >> 2), tlB = tlA + 8;     // TMEM lanes of the two rows
+    const int rowA = 4 * (tlA - quarter * 32) + quarter, rowB = rowA + 32;   // query rows within the tile
     const uint32_t tS0 = tmem + ((uint32_t)(quarter * 32 + half * 16) << 16);
     const uint32_t tO16 = tS0 + 384;
-    // epilogue: 32x32b, thread = row quarter*32 + lane, O columns half*64 .. +63
-    const int row = quarter * 32 + lane;
+    // epilogue: 32x32b, thread = TMEM lane quarter*32 + lane (query row
+    // 4 lane + quarter), O columns half*64 .. +63
+    const int row = 4 * lane + quarter;
     const uint32_t tO = tmem + ((uint32_t)(quarter * 32) << 16) + 384 + half * 64;
     float* xsum = reinterpret_cast<float*>(smem + OFF_XCHG);    // [item parity][row]
     const float c = p.scale_log2;
@@ -656,10 +669,27 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_fwd_kernel(const __gr
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(B_SLEMPTY + sl));
       const int qtA = M.q0 + rowA, qtB = M.q0 + rowB;
+      // a warp whose 16 rows are all past the chunk's end does no softmax work
+      // (the P of its lanes only feeds O rows that are never stored)
+      const bool idle = 64 * half + quarter >= M.q_rows;
       float mA = -INFINITY, mB = -INFINITY, lA = 0.f, lB = 0.f;
       bool ok = true;
       for (int kt = 0; kt < M.T; ++kt, ++g) {
         const int sb = g % NSB, tk = g % NTOK;
+        if (idle) {
+          // S(g) complete implies both barriers' previous phases completed, so
+          // these arrives count toward tile g
+          if (!fl.wait(bar(B_SFULL + sb), (g / NSB) & 1) || !fl.wait(bar(B_TOKFULL + tk), (g / NTOK) & 1)) {
+            ok = false;
+            break;
+          }
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive(bar(B_TOKEMPTY + tk));
+            mbar_arrive(bar(B_PREADY + sb));
+          }
+          continue;
+        }
         // both barriers tested back to back (the usual case: both complete)
         const bool s_done = mbar_test_wait(bar(B_SFULL + sb), (g / NSB) & 1);
         const bool t_done = mbar_test_wait(bar(B_TOKFULL + tk), (g / NTOK) & 1);
@@ -792,13 +822,13 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_fwd_kernel(const __gr
       lB += __shfl_xor_sync(0xffffffffu, lB, 2);
       const int lb = n_local & 1;
       if (cq == 0) {
-        xsum[lb * BM + rowA] = lA;
-        xsum[lb * BM + rowB] = lB;
+        xsum[lb * BM + tlA] = lA;
+        xsum[lb * BM + tlB] = lB;
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(B_XSUM + quarter * 2 + lb));
       if (!fl.wait(bar(B_XSUM + quarter * 2 + lb), (n_local >> 1) & 1)) break;
-      const float l_tot = xsum[lb * BM + row];
+      const float l_tot = xsum[lb * BM + quarter * 32 + lane];
       if (!fl.wait(bar(B_OFINAL), n_local & 1)) break;
       tc_fence_after();
       const float inv_l = M.T > 0 ? 1.f / l_tot : 0.f;
@@ -858,7 +888,15 @@ int launch_sparse_attn_long(const AttnWork& w, const void* Q, const void* K, con
   if (!enc) return cuda_status(cudaErrorNotSupported);
   AttnMaps maps;
   const long long q_rows = (long long)B * Hq * L, kv_rows = (long long)B * Hkv * L;
-  bool ok = make_rows_map(enc, &maps.q, Q, q_rows, BM);
+  // Q as four views of every fourth row (residues 0..3); an empty residue
+  // class (fewer than four rows in all) reuses view 0
+  bool ok = true;
+  for (int r = 0; r < 4; ++r) {
+    const long long n_r = (q_rows - r + 3) / 4;
+    const int src = n_r > 0 ? r : 0;
+    ok = ok && make_rows_view_map(enc, &maps.q[r], reinterpret_cast<const __nv_bfloat16*>(Q) + (long long)src * kHeadDim,
+                                  n_r > 0 ? n_r : (q_rows + 3) / 4, 4, 32);
+  }
   for (int s = 0; s < 16; ++s) {
     ok = ok && make_rows_map(enc, &maps.k[s], K, kv_rows, 8 * (s + 1));
     ok = ok && make_rows_map(enc, &maps.v[s], V, kv_rows, 8 * (s + 1));

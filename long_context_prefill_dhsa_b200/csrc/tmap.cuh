@@ -38,6 +38,20 @@ inline bool make_rows_map(EncodeTiledFn enc, CUtensorMap* m, const void* base, l
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// A view of every `step`-th row of a [rows_total, kHeadDim] bf16 tensor,
+// starting at `base`: view row y is base row step*y. Rows past `rows` read
+// as zeros.
+inline bool make_rows_view_map(EncodeTiledFn enc, CUtensorMap* m, const void* base, long long rows, int step,
+                               int box_rows) {
+  const cuuint64_t dims[2] = {(cuuint64_t)kHeadDim, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)kHeadDim * 2 * step};
+  const cuuint32_t box[2] = {64u, (cuuint32_t)box_rows};
+  const cuuint32_t estr[2] = {1u, 1u};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Work lists of the two attention kernels (built on the device by
 // launch_build_items). Long items are (b, hq, chunk, 128-row tile index),
 // short items (b, hq, chunk, first row of the tile within the chunk).
