@@ -39,6 +39,10 @@ SMALL = {
     "k-all-dense": I.custom(B=2, Hq=4, Hkv=2, L=640, lo=5, hi=60, k=100000, wid=105),
     "single-chunk": I.custom(B=1, Hq=2, Hkv=1, L=200, lo=500, hi=600, k=3, wid=106),
     "short-seq": I.custom(B=3, Hq=2, Hkv=1, L=37, lo=1, hi=9, k=2, wid=107),
+    # fewer than four Q rows in all: the attention loads Q through four views
+    # of every fourth row, and these leave some views empty
+    "three-rows": I.custom(B=1, Hq=1, Hkv=1, L=3, lo=1, hi=2, k=2, wid=116),
+    "one-row": I.custom(B=1, Hq=1, Hkv=1, L=1, lo=1, hi=2, k=2, wid=117),
     "geometric": I.custom(B=2, Hq=4, Hkv=1, L=3000, lo=1, hi=1024, kind="geometric", mean=40.0, k=6, wid=108),
 }
 
