@@ -23,9 +23,12 @@
 // * Masking: padding slots are removed inside the tensor core. Every QK^T
 //   gets one extra K=16 MMA step, ones-column x per-slot bias (0 for a kept
 //   key, -inf for a padding slot), so S already holds -inf there. Only tiles
-//   that hold keys of the diagonal chunk past the tile's first query row
-//   mask causally: that piece is the tile's last and its slots hold
-//   consecutive tokens, so a row masks the slots from one threshold on.
+//   that hold keys of the diagonal chunk mask causally: that chunk is the
+//   key stream's last and its slots hold consecutive tokens, so a row masks
+//   the slots from one threshold on. Every chunk takes round8(length)
+//   consecutive stream slots, so the scheduler gives the diagonal chunk's
+//   first slot with the item and the softmax computes each row's threshold
+//   itself.
 // * Warp roles (512 threads, four warpgroups): warp 0 = TMA producer of Q
 //   and K (and of the bias blocks), warp 3 = TMA producer of V, warp 1 =
 //   QK^T issuer, warp 14 = PV issuer (one thread each), warp 2 = scheduler
@@ -88,7 +91,6 @@ constexpr int BN = 128;              // key slots per tile
 constexpr int NSK = 2;               // K pipeline stages
 constexpr int NSV = 2;               // V pipeline stages
 constexpr int NSB = 3;               // S/P buffers in TMEM
-constexpr int NTOK = 4;              // slot-token table ring (causal tiles)
 constexpr int NSLOT = 4;             // scheduled work items in flight
 constexpr int SEG_CAP = 64;          // chunk descriptors kept in shared memory per item
 constexpr int kThreads = 512;
@@ -131,7 +133,8 @@ struct ItemMeta {
   int b;
   int i;         // query chunk
   int c_start;   // first token of chunk i
-  int pad[2];
+  int diag_slot; // key-stream slot where the diagonal chunk starts
+  int pad;
 };
 struct ItemSlot {
   ItemMeta m;
@@ -144,8 +147,7 @@ constexpr uint32_t OFF_K = OFF_Q + 2 * kTileBytes;              // NSK x 32 KB
 constexpr uint32_t OFF_V = OFF_K + NSK * kTileBytes;            // NSV x 32 KB
 constexpr uint32_t OFF_ONES = OFF_V + NSV * kTileBytes;         // 4 KB
 constexpr uint32_t OFF_BIAS = OFF_ONES + kBiasBytes;            // NSK x 4 KB
-constexpr uint32_t OFF_TINFO = OFF_BIAS + NSK * kBiasBytes;    // NTOK int4 tile descriptors
-constexpr uint32_t OFF_SLOT = OFF_TINFO + NTOK * 16;
+constexpr uint32_t OFF_SLOT = OFF_BIAS + NSK * kBiasBytes;
 constexpr uint32_t OFF_XCHG = OFF_SLOT + NSLOT * sizeof(ItemSlot);   // row sums, [item parity][row]
 constexpr uint32_t OFF_BAR = OFF_XCHG + 2 * BM * 4;
 enum {
@@ -155,9 +157,7 @@ enum {
   B_SLEMPTY = B_SLFULL + NSLOT,
   B_KFULL = B_SLEMPTY + NSLOT,
   B_VFULL = B_KFULL + NSK,
-  B_TOKFULL = B_VFULL + NSV,
-  B_TOKEMPTY = B_TOKFULL + NTOK,
-  B_SFULL = B_TOKEMPTY + NTOK,   // QK^T(g) complete: S ready, K stage and bias block free
+  B_SFULL = B_VFULL + NSV,   // QK^T(g) complete: S ready, K stage and bias block free
   B_PREADY = B_SFULL + NSB,
   B_PVDONE = B_PREADY + NSB,     // PV(g) complete: P buffer and V stage free, O current
   B_OFINAL = B_PVDONE + NSB,
@@ -286,8 +286,6 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_fwd_kernel(const __gr
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
-  // per key tile: (causal, first slot of the diagonal piece, that slot minus its token)
-  int4* tile_info = reinterpret_cast<int4*>(smem + OFF_TINFO);
   ItemSlot* slots = reinterpret_cast<ItemSlot*>(smem + OFF_SLOT);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_ABORT);
   auto bar = [&](int idx) { return sbase + OFF_BAR + 8u * idx; };
@@ -314,10 +312,6 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_fwd_kernel(const __gr
       }
       for (int s = 0; s < NSK; ++s) mbar_init(bar(B_KFULL + s), 1);
       for (int s = 0; s < NSV; ++s) mbar_init(bar(B_VFULL + s), 1);
-      for (int s = 0; s < NTOK; ++s) {
-        mbar_init(bar(B_TOKFULL + s), 1);
-        mbar_init(bar(B_TOKEMPTY + s), kSoftmaxWarps);
-      }
       mbar_init(bar(B_OFINAL), 1);
       mbar_init(bar(B_FINAL), 1);
       mbar_init(bar(B_FINALPV), 1);
@@ -338,7 +332,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_fwd_kernel(const __gr
   // get -inf added; a masked V row is multiplied by P = 0): zero every K and
   // V stage and the bias blocks once; then write the ones column of the bias
   // step's A operand.
-  for (uint32_t o = threadIdx.x * 16; o < OFF_TINFO - OFF_K; o += kThreads * 16)
+  for (uint32_t o = threadIdx.x * 16; o < OFF_SLOT - OFF_K; o += kThreads * 16)
     *reinterpret_cast<uint4*>(smem + OFF_K + o) = make_uint4(0, 0, 0, 0);
   __syncthreads();
   if (threadIdx.x < BM) *reinterpret_cast<uint16_t*>(smem + OFF_ONES + noswz_off(threadIdx.x, 0)) = kBf16One;
@@ -385,16 +379,22 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_fwd_kernel(const __gr
       const long long r = ((long long)b * p.Hq + hq) * p.Nmax + i;
       const int rp0 = p.row_ptr[r], rp1 = p.row_ptr[r + 1];
       ItemSlot& S = slots[sl];
-      int nslots = 0;
+      // every chunk takes round8(len) consecutive key-stream slots (a piece
+      // split at a tile boundary continues at slot 0 of the next tile)
+      int nslots = 0, last = 0;
       for (int q = rp0 + lane; q < rp1; q += 32) {
         const int j = min(max(p.col_idx[q], 0), i);   // a bad index cannot leave the offsets row
         const int s0 = ob[j];
         const int len = (j == i) ? (q0 + q_rows - c_start) : (ob[j + 1] - s0);
         nslots += round8(len);
+        if (q == rp1 - 1) last = round8(len);
         if (q - rp0 < SEG_CAP) S.seg[q - rp0] = make_int2(s0, len);
       }
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) nslots += __shfl_xor_sync(0xffffffffu, nslots, o);
+      for (int o = 16; o > 0; o >>= 1) {
+        nslots += __shfl_xor_sync(0xffffffffu, nslots, o);
+        last += __shfl_xor_sync(0xffffffffu, last, o);
+      }
       if (lane == 0) {
         S.m.q0 = q0;
         S.m.q_rows = q_rows;
@@ -406,6 +406,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_fwd_kernel(const __gr
         S.m.b = b;
         S.m.i = i;
         S.m.c_start = c_start;
+        S.m.diag_slot = nslots - last;   // the diagonal chunk is the row's last
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(B_SLFULL + sl));
@@ -460,11 +461,11 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_fwd_kernel(const __gr
       int sq = 0, seg_pos = 0;
       bool ok = true;
       for (int kt = 0; kt < M.T; ++kt, ++g) {
-        const int stk = g % NSK, stv = g % NSV, tk = g % NTOK;
+        const int stk = g % NSK, stv = g % NSV;
         // walk the key stream of this tile first, in registers only (the
         // stage waits below then overlap it): lane b holds the b-th TMA box,
         // and bit i of kept the state of slot lane + 32 i
-        int slot = 0, causal = 0, d_slot = 0, d_off = 0, nbox = 0, my_y = 0, my_so = 0, my_bx = 0;
+        int slot = 0, nbox = 0, my_y = 0, my_so = 0, my_bx = 0;
         uint32_t bytes = 0, kept = 0;
         while (slot < BN && sq < M.nseg) {
           const int2 dsc = desc(sq);
@@ -477,13 +478,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_fwd_kernel(const __gr
               const int s = lane + 32 * q;
               if (s >= slot && s < slot + rows) kept |= 1u << q;
             }
-            if (sq == M.nseg - 1 && tok0 + rows - 1 > M.q0) {
-              // diagonal keys past the first query: the piece is the tile's
-              // last, slot s >= d_slot holds token s - d_off
-              causal = 1;
-              d_slot = slot;
-              d_off = slot - tok0;
-            }
+
           }
           // the whole piece in one box per head-dim half (per-op TMA cost
           // dominates for small boxes, so never split a piece)
@@ -504,7 +499,6 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_fwd_kernel(const __gr
         if (kprod) {
           // the K stage (and its bias block) of tile g - NSK is free once that QK^T is done
           if (g >= NSK && !fl.wait(bar(B_SFULL + (g - NSK) % NSB), ((g - NSK) / NSB) & 1)) { ok = false; break; }
-          if (g >= NTOK && !fl.wait(bar(B_TOKEMPTY + tk), ((g / NTOK) - 1) & 1)) { ok = false; break; }
           // copies first; the bias block and the tile descriptor follow, and
           // the stage's barrier completes only after this warp's arrive
           if (lane == 0) mbar_expect_tx(bar(B_KFULL + stk), bytes);
@@ -518,11 +512,9 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_fwd_kernel(const __gr
 #pragma unroll
           for (int q = 0; q < 4; ++q)
             *reinterpret_cast<uint16_t*>(bias + noswz_off(lane + 32 * q, 0)) = ((kept >> q) & 1u) ? 0 : kBf16NegInf;
-          if (lane == 0) tile_info[tk] = make_int4(causal, d_slot, d_off, 0);
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
-            mbar_arrive(bar(B_TOKFULL + tk));
             mbar_arrive(bar(B_KFULL + stk));
           }
         } else {
@@ -675,26 +667,19 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_fwd_kernel(const __gr
       float mA = -INFINITY, mB = -INFINITY, lA = 0.f, lB = 0.f;
       bool ok = true;
       for (int kt = 0; kt < M.T; ++kt, ++g) {
-        const int sb = g % NSB, tk = g % NTOK;
+        const int sb = g % NSB;
         if (idle) {
-          // S(g) complete implies both barriers' previous phases completed, so
-          // these arrives count toward tile g
-          if (!fl.wait(bar(B_SFULL + sb), (g / NSB) & 1) || !fl.wait(bar(B_TOKFULL + tk), (g / NTOK) & 1)) {
+          // S(g) complete implies PREADY's phase of tile g - NSB completed, so
+          // this arrive counts toward tile g
+          if (!fl.wait(bar(B_SFULL + sb), (g / NSB) & 1)) {
             ok = false;
             break;
           }
           __syncwarp();
-          if (lane == 0) {
-            mbar_arrive(bar(B_TOKEMPTY + tk));
-            mbar_arrive(bar(B_PREADY + sb));
-          }
+          if (lane == 0) mbar_arrive(bar(B_PREADY + sb));
           continue;
         }
-        // both barriers tested back to back (the usual case: both complete)
-        const bool s_done = mbar_test_wait(bar(B_SFULL + sb), (g / NSB) & 1);
-        const bool t_done = mbar_test_wait(bar(B_TOKFULL + tk), (g / NTOK) & 1);
-        if (!(s_done && t_done) &&
-            (!fl.wait(bar(B_SFULL + sb), (g / NSB) & 1) || !fl.wait(bar(B_TOKFULL + tk), (g / NTOK) & 1))) {
+        if (!fl.wait(bar(B_SFULL + sb), (g / NSB) & 1)) {
           ok = false;
           break;
         }
@@ -704,10 +689,12 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_fwd_kernel(const __gr
         tmem_ld_16x256b_x8(tS0 + sb * 128 + 0, *reinterpret_cast<uint32_t(*)[32]>(s + 0));
         tmem_ld_16x256b_x8(tS0 + sb * 128 + 64, *reinterpret_cast<uint32_t(*)[32]>(s + 32));
         tmem_wait_ld();
-        const int4 ti = tile_info[tk];
-        if (ti.x) {
-          // keys after the query token: the slots from the row's threshold on
-          const int thrA = max(qtA + ti.z + 1, ti.y), thrB = max(qtB + ti.z + 1, ti.y);
+        // the diagonal chunk, the key stream's last, starts at slot dt of this
+        // tile (dt < 0: in an earlier tile) and its slot s holds token
+        // c_start + s - dt: a row masks the slots from qt - c_start + dt + 1 on
+        const int dt = M.diag_slot - BN * kt;
+        if (dt < BN) {
+          const int thrA = max(qtA - M.c_start + dt + 1, 0), thrB = max(qtB - M.c_start + dt + 1, 0);
 #pragma unroll
           for (int j = 0; j < 16; ++j)
 #pragma unroll
@@ -717,8 +704,6 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_fwd_kernel(const __gr
               if (col >= thrB) s[4 * j + 2 + e] = __float_as_uint(-INFINITY);
             }
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(B_TOKEMPTY + tk));
         // row maxima: two chains per row over the thread's 32 columns
         auto S = [&](int e) { return __uint_as_float(s[e]); };
         float a0 = fmaxf(S(0), S(1)), a1 = fmaxf(S(4), S(5));
